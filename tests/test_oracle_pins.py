@@ -1,0 +1,293 @@
+"""Pins of the fp64 oracle against what the pages and mathematics fix.
+
+No page prints a worked value, so each step is pinned by closed forms,
+invariants, special cases that reduce to a textbook routine, and brute force on
+tiny inputs -- chosen so that a dropped term, a wrong sign or index or a
+transposed operand in the oracle fails at least one of them.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from cluster_guided_sparse_b200 import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------- RoPE
+def test_rope_hand_examples():
+    g = _gold("rope_pairs.json")
+    T, Hh, W = g["grid"]
+    N, D = T * Hh * W, sum(g["d_split"])
+    for case in g["cases"]:
+        x = np.zeros((N, D))
+        x[case["token"]] = case["x"]
+        y = oracle.rope3d(x, g["grid"], g["d_split"], g["theta"])
+        np.testing.assert_allclose(y[case["token"]], case["expect"], rtol=0, atol=1e-15, err_msg=case["note"])
+
+
+def test_rope_norm_and_identity_at_origin():
+    rng = np.random.default_rng(1)
+    grid, ds = (3, 4, 5), (8, 12, 12)
+    x = rng.standard_normal((60, 32))
+    y = oracle.rope3d(x, grid, ds, 10000.0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    np.testing.assert_array_equal(y[0], x[0])
+    # per-pair norms are kept too (each pair is a plane rotation)
+    np.testing.assert_allclose(np.hypot(y[:, 0::2], y[:, 1::2]), np.hypot(x[:, 0::2], x[:, 1::2]), rtol=1e-12)
+
+
+def test_rope_relative_position_invariance():
+    """<R_{m+s} q, R_{n+s} k> = <R_m q, R_n k> for any per-axis shift s."""
+    rng = np.random.default_rng(2)
+    grid, ds = (6, 7, 9), (8, 12, 12)
+    T, Hh, W = grid
+    D = sum(ds)
+    q, k = rng.standard_normal(D), rng.standard_normal(D)
+
+    def tok(t, y, x):
+        return (t * Hh + y) * W + x
+
+    for (m, n, s) in [((0, 1, 2), (3, 4, 5), (1, 2, 3)), ((2, 0, 8), (0, 6, 0), (3, 0, 0)),
+                      ((1, 1, 1), (1, 1, 1), (4, 5, 7))]:
+        X = np.zeros((T * Hh * W, D))
+        a, b = tok(*m), tok(*n)
+        a2 = tok(*(mi + si for mi, si in zip(m, s)))
+        b2 = tok(*(ni + si for ni, si in zip(n, s)))
+        X[a], X[a2] = q, q
+        Y = oracle.rope3d(X, grid, ds, 10000.0)
+        Xk = np.zeros_like(X)
+        Xk[b], Xk[b2] = k, k
+        Yk = oracle.rope3d(Xk, grid, ds, 10000.0)
+        assert abs(Y[a] @ Yk[b] - Y[a2] @ Yk[b2]) < 1e-12 * (np.linalg.norm(q) * np.linalg.norm(k))
+
+
+def test_rope_no_grid_is_identity():
+    x = np.random.default_rng(3).standard_normal((16, 8))
+    np.testing.assert_array_equal(oracle.rope3d(x, (0, 0, 0), (8, 0, 0), 10000.0), x)
+
+
+# ----------------------------------------------------------------------------- k-means
+def test_kmeans_brute_force_assign_and_ties():
+    rng = np.random.default_rng(4)
+    x = rng.integers(-3, 4, size=(200, 3)).astype(float)
+    c = rng.integers(-3, 4, size=(7, 3)).astype(float)
+    lab = oracle.kmeans_assign(x, c)
+    for n in range(x.shape[0]):
+        d = [sum((x[n, t] - c[j, t]) ** 2 for t in range(3)) for j in range(7)]
+        best = min(d)
+        assert lab[n] == d.index(best)  # first (lowest) index among the minima
+    # an equidistant point goes to the lower index
+    assert oracle.kmeans_assign(np.array([[0.0, 0.0]]), np.array([[1.0, 0.0], [-1.0, 0.0]]))[0] == 0
+    assert oracle.kmeans_assign(np.array([[0.0, 0.0]]), np.array([[5.0, 0.0], [0.0, 1.0], [1.0, 0.0]]))[0] == 1
+
+
+def test_kmeans_objective_never_increases():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((500, 6)) + rng.integers(0, 4, size=(500, 1)) * 3.0
+    C = 9
+    cent = x[np.arange(C) * (500 // C)].copy()
+    prev = np.inf
+    for _ in range(8):
+        lab = oracle.kmeans_assign(x, cent)
+        J_assign = oracle.kmeans_objective(x, lab, cent)
+        assert J_assign <= prev + 1e-9
+        cent, _ = oracle.kmeans_update(x, lab, cent)
+        J_update = oracle.kmeans_objective(x, lab, cent)
+        assert J_update <= J_assign + 1e-9
+        prev = J_update
+
+
+def test_kmeans_separated_blobs_recover_means():
+    """Strided init picks one point per blob -> blob means after one update."""
+    rng = np.random.default_rng(6)
+    C, per, D = 4, 25, 5
+    centers = np.eye(C, D) * 100.0
+    x = np.concatenate([centers[j] + rng.standard_normal((per, D)) for j in range(C)])
+    lab, cent, sizes = oracle.kmeans(x, C, iters=1)
+    for j in range(C):
+        np.testing.assert_allclose(cent[j], x[j * per:(j + 1) * per].mean(0), rtol=0, atol=1e-12)
+        assert (lab[j * per:(j + 1) * per] == j).all()
+    assert sizes.tolist() == [per] * C
+
+
+def test_kmeans_init_offset_and_empty_cluster():
+    x = np.array([[0.0], [1.0], [2.0], [3.0], [100.0], [101.0]])
+    # strided init with stride 3 and seed 1 -> offset 1: centroids x[1], x[4]
+    lab, cent, _ = oracle.kmeans(x, 2, iters=0, seed=1)
+    np.testing.assert_array_equal(cent[:, 0], [1.0, 100.0])
+    assert lab.tolist() == [0, 0, 0, 0, 1, 1]
+    # a centroid far from every point gets no member and keeps its place
+    c0 = np.array([[0.0], [1000.0], [101.0]])
+    l0 = oracle.kmeans_assign(x, c0)
+    c1, sizes = oracle.kmeans_update(x, l0, c0)
+    assert sizes[1] == 0 and c1[1, 0] == 1000.0
+    np.testing.assert_allclose(c1[:, 0], [1.5, 1000.0, 100.5])
+
+
+# ----------------------------------------------------------------------------- LUT / proxy
+def test_lut_sum_is_product_quantised_dot():
+    """s_c(j) = qbar_c . concat(mu_t[a_t(j)], mu_h[a_h(j)], mu_w[a_w(j)])."""
+    rng = np.random.default_rng(7)
+    ds, Cs, Cq, N = (4, 6, 6), (3, 5, 4), 6, 40
+    qc = rng.standard_normal((Cq, sum(ds)))
+    offs = np.cumsum((0,) + ds)
+    kcs = [rng.standard_normal((Cs[s], ds[s])) for s in range(3)]
+    codes = [rng.integers(0, Cs[s], N).astype(np.int32) for s in range(3)]
+    luts = [oracle.lut(qc[:, offs[s]:offs[s + 1]], kcs[s]) for s in range(3)]
+    for c in range(Cq):
+        s = oracle.proxy_scores([L[c] for L in luts], codes)
+        full = np.stack([np.concatenate([kcs[t][codes[t][j]] for t in range(3)]) for j in range(N)])
+        np.testing.assert_allclose(s, full @ qc[c], rtol=1e-13, atol=1e-13)
+
+
+def test_each_key_its_own_centroid_gives_exact_per_query_topp():
+    """C_q = C_t = C_h = C_w = N: proxy = exact q.k, so selection = exact Top-p per query."""
+    w, (q, k, v) = synth.tiny_case(N=32, D=8, grid=(2, 4, 4), d_split=(2, 2, 4), c_q=32, c_sub=(32, 32, 32), k_min=0)
+    p = oracle.Params.of(w)
+    q0, k0 = q[0, 0].double().numpy(), k[0, 0].double().numpy()
+    out = oracle.scope_plan_head(q0, k0, p)
+    assert (out["q_labels"] == np.arange(32)).all()
+    assert all((c == np.arange(32)).all() for c in out["codes"])
+    logits = out["qr"] @ out["kr"].T / np.sqrt(8)
+    for i in range(32):
+        o = np.lexsort((np.arange(32), -logits[i]))
+        wgt = np.exp(logits[i] - logits[i].max())
+        cum = np.cumsum(wgt[o]) / wgt.sum()
+        m = int(np.argmax(cum >= p.top_p - 1e-15)) + 1
+        assert out["r"][i] == min(32, max(m, p.k_min))
+
+
+# ----------------------------------------------------------------------------- Top-p
+def test_topp_brute_force_minimal_set():
+    rng = np.random.default_rng(8)
+    for trial in range(60):
+        N = int(rng.integers(1, 11))
+        s = rng.integers(-3, 4, N).astype(float) * rng.choice([0.5, 1.0, 3.0])
+        p = float(rng.choice([0.3, 0.5, 0.8, 0.9, 0.99]))
+        scale = 1.0
+        w = np.exp(s - s.max())
+        m = oracle.topp_count(s, p, scale)
+        sel = set(oracle.emit(s, m).tolist())
+        assert len(sel) == m
+        # the chosen set reaches p, no smaller set does
+        assert w[list(sel)].sum() >= p * w.sum() - 1e-12
+        for size in range(m):
+            for sub in itertools.combinations(range(N), size):
+                assert w[list(sub)].sum() < p * w.sum() + 1e-12
+        # among equal scores the lower index wins: the set is the lexicographic
+        # first of the best-mass sets of size m
+        best = max(itertools.combinations(range(N), m), key=lambda sub: (round(w[list(sub)].sum(), 12), [-i for i in sub]))
+        assert sel == set(best)
+
+
+def test_topp_uniform_closed_form():
+    for N, p, m in [(256, 0.9, 231), (256, 0.5, 128), (128, 0.25, 32), (64, 0.999, 64)]:
+        assert oracle.topp_count(np.zeros(N), p, 1.0) == m
+    assert oracle.topp_count(np.arange(10.0), 1.0, 1.0) == 10
+
+
+def test_topp_dominant_key():
+    s = np.array([0.0, 0.0, 50.0, 0.0])
+    assert oracle.topp_count(s, 0.9, 1.0) == 1
+    assert oracle.emit(s, 1).tolist() == [2]
+    assert oracle.retained_count(s, 0.9, 3, 1.0) == 3
+    assert oracle.emit(s, 3).tolist() == [0, 1, 2]  # ties at 0.0 go to the lowest indices
+
+
+# ----------------------------------------------------------------------------- online Top-k
+def test_online_topk_hand_examples():
+    g = _gold("online_topk.json")
+    for case in g["cases"]:
+        K, n = oracle.online_topk(case["sizes"], case["r"], case["N"], online=True)
+        assert K == case["K_h"], case["work"]
+        assert n.tolist() == case["n"], case["work"]
+    K, n = oracle.online_topk([5, 2, 1], [10, 4, 3], 1000, online=False)
+    assert n.tolist() == [10, 4, 3]
+
+
+# ----------------------------------------------------------------------------- attention
+def test_full_selection_equals_dense_attention():
+    rng = np.random.default_rng(9)
+    N, D = 40, 16
+    qr, kr, v = (rng.standard_normal((N, D)) * 2 for _ in range(3))
+    lab = np.zeros(N, np.int32)
+    o = oracle.scope_attn_head(qr, kr, v, lab, [np.arange(N, dtype=np.int32)])
+    # independent dense reference: explicit softmax rows
+    ref = np.empty_like(o)
+    for i in range(N):
+        lg = np.array([qr[i] @ kr[j] for j in range(N)]) / 4.0
+        e = np.exp(lg - lg.max())
+        ref[i] = (e / e.sum()) @ v
+    np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(oracle.dense_attention(qr, kr, v), ref, rtol=0, atol=1e-12)
+
+
+def test_attention_equal_logits_and_single_key():
+    rng = np.random.default_rng(10)
+    K, V = rng.standard_normal((10, 4)), rng.standard_normal((10, 4))
+    sel = np.array([1, 4, 7], np.int32)
+    o = oracle.attention_rows(np.zeros((1, 4)), K, V, sel, 0.5)
+    np.testing.assert_allclose(o[0], V[sel].mean(0), atol=1e-15)
+    o = oracle.attention_rows(rng.standard_normal((2, 4)), K, V, np.array([6], np.int32), 0.5)
+    np.testing.assert_allclose(o, V[[6, 6]], atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- bisection
+def test_bisect_balanced_leaves_and_first_split():
+    rng = np.random.default_rng(11)
+    N, D, leaf = 512, 8, 64
+    blob = np.where(rng.permutation(N) < N // 2, 1.0, -1.0)
+    x = rng.standard_normal((N, D)) + blob[:, None] * 50.0
+    lab, cent, perm = oracle.bisect(x, leaf, 10)
+    assert np.bincount(lab).tolist() == [leaf] * (N // leaf)
+    assert sorted(perm.tolist()) == list(range(N))
+    for c in range(N // leaf):
+        members = perm[c * leaf:(c + 1) * leaf]
+        assert (lab[members] == c).all()
+        assert (np.diff(members) > 0).all()  # token order within a leaf
+        np.testing.assert_allclose(cent[c], x[members].mean(0), atol=1e-12)
+    first = lab < (N // leaf) // 2
+    assert (blob[first] == blob[first][0]).all() and (blob[~first] == -blob[first][0]).all()
+    with pytest.raises(ValueError):
+        oracle.bisect(x[:448], leaf, 10)  # 7 leaves: not a power of two
+
+
+def test_bisect_median_split_ties_by_token():
+    # points on a line: the lower half of delta (closer to c0) goes to child 0
+    x = np.array([[0.0], [10.0], [1.0], [9.0], [2.0], [8.0], [3.0], [7.0]])
+    lab, _, _ = oracle.bisect(x, 4, 3)
+    assert lab.tolist() == [0, 1, 0, 1, 0, 1, 0, 1]
+    # all points equal: every delta ties, so the split is by token index
+    lab, _, _ = oracle.bisect(np.ones((8, 2)), 2, 2)
+    assert lab.tolist() == [0, 0, 1, 1, 2, 2, 3, 3]
+
+
+# ----------------------------------------------------------------------------- pipeline
+def test_pipeline_tiny_config_invariants():
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.make_inputs(w)
+    p = oracle.Params.of(w)
+    for h in range(w.H):
+        out = oracle.scope_plan_head(q[0, h].double().numpy(), k[0, h].double().numpy(), p)
+        N = w.N
+        assert out["q_sizes"].sum() == N
+        assert (out["r"] >= min(N, p.k_min)).all() and (out["r"] <= N).all()
+        nonempty = out["q_sizes"] > 0
+        K = -(-int((out["q_sizes"] * out["r"]).sum()) // N)
+        assert out["K_h"] == K
+        assert (out["n"][nonempty] >= np.maximum(out["r"][nonempty], K).clip(max=N)).all()
+        for c, lst in enumerate(out["lists"]):
+            assert len(lst) == out["n"][c]
+            assert (np.diff(lst) > 0).all()
+        o = oracle.scope_attn_head(out["qr"], out["kr"], v[0, h].double().numpy(), out["q_labels"], out["lists"])
+        assert np.isfinite(o).all()
