@@ -1,0 +1,107 @@
+// Internal declarations shared by the libscope.so translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace scope {
+
+constexpr int kSortBlk = 512;   // points per warp-block in the stable label sort
+constexpr int kMaxClusters = 1024;
+constexpr int kTQ = 128;        // query rows per attention tile
+constexpr int kMaxItems = 65536; // c_t * c_h * c_w bound (distinct code triples)
+
+// Device error word bits (workspace int32[4]).
+constexpr int kErrRange = 1;
+constexpr int kErrTimeout = 2;
+
+// One clustering problem: rows X[bh][n][dim_off : dim_off + dim_n] into C
+// clusters.  Key subspaces and queries of one plan run as one batch.
+struct KmProblem {
+    const __nv_bfloat16 *X;     // [BH][N][D]
+    const uint32_t *maxabs;     // bits of max |X| (non-negative float), set by RoPE
+    int dim_off, dim_n, C;
+    int32_t *labels;            // [BH][N]
+    float *cent;                // [BH][C][dim_n]
+    float *cn;                  // [BH][C] squared centroid norms
+    int32_t *sizes;             // [BH][C]
+    int32_t *perm;              // [BH][N]   members cluster by cluster, ascending
+    int32_t *start;             // [BH][C+1] cluster starts in perm
+    int32_t *blockhist;         // [BH][C][nblk]
+};
+
+struct KmBatch {
+    KmProblem p[4];
+    int count;
+};
+
+// Count of kernels launched by the library (see scope_kernel_launches).
+void count_launches(int n);
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ uint32_t ordered_key(float s)
+{
+    // Monotone map float -> uint32: larger float -> larger key (no NaNs here).
+    uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt()
+{
+    uint32_t m;
+    asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_incl_scan(T v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        T t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+
+// Block-wide exclusive scan (blockDim.x a multiple of 32, <= 1024).
+// `tmp` needs 33 elements of shared memory.  Returns the exclusive prefix;
+// `total` receives the block sum.  Deterministic (fixed combination order).
+template <typename T>
+__device__ __forceinline__ T block_excl_scan(T v, T *tmp, T &total)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    T inc = warp_incl_scan(v);
+    __syncthreads();
+    if (lane == 31) tmp[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        T w = lane < nw ? tmp[lane] : T(0);
+        T wi = warp_incl_scan(w);
+        if (lane < nw) tmp[lane] = wi - w;
+        if (lane == nw - 1) tmp[32] = wi;
+    }
+    __syncthreads();
+    total = tmp[32];
+    return tmp[wid] + inc - v;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_max(T v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ void set_error(int32_t *err, int bit, int detail)
+{
+    if (err) {
+        atomicOr(err, bit);
+        atomicCAS(err + 1, 0, detail);
+    }
+}
+
+}  // namespace scope

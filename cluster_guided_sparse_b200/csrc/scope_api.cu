@@ -1,0 +1,574 @@
+// Host side of libscope.so: argument checks, workspace layout, the launch
+// sequence of scope_plan / scope_attn / scope_dense_attn, result views.
+// Every argument check runs before any CUDA call, so a bad call never
+// touches the device.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <atomic>
+#include <string>
+
+#include "../../include/scope.h"
+#include "common.cuh"
+
+namespace scope {
+// kernels.cu launchers
+void launch_rope_table(double2 *, int, int, int, int, int, int, double, int, int, cudaStream_t);
+void launch_rope_apply(const void *, bool, __nv_bfloat16 *, float *, uint32_t *, const double2 *, int64_t, int, int,
+                       int, int, int, int, int, int, int, cudaStream_t);
+void launch_to_bf16(const float *, __nv_bfloat16 *, int64_t, cudaStream_t);
+cudaError_t km_configure();
+void launch_km_init(const KmBatch &, int, int, int, uint32_t, cudaStream_t);
+void launch_km_assign_direct(const KmBatch &, int, int, int, cudaStream_t);
+void launch_km_sort(const KmBatch &, int, int, cudaStream_t);
+void launch_km_reduce(const KmBatch &, int, int, int, cudaStream_t);
+struct SelArgs;
+void launch_lut(const float *, const float *, const float *, const float *, float *, int, int, int, int, int, int,
+                int, int, int, cudaStream_t);
+void launch_items(const int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, int, int, int, int, int, int,
+                  cudaStream_t);
+void launch_tiles(const int32_t *, int2 *, int32_t *, int, int, int, cudaStream_t);
+void launch_attn_simt(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, __nv_bfloat16 *,
+                      const int2 *, const int32_t *, int, const int32_t *, const int32_t *, const long long *,
+                      const int32_t *, const int32_t *, int, int, int, int, cudaStream_t);
+void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
+                   const int32_t *item_n, int Pcap, int N, int Cq, int Ct, int Ch, int Cw, int BH, float top_p,
+                   float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes, int32_t *r, int32_t *n,
+                   int32_t *kh, long long *offsets, int32_t *indices, int online, cudaStream_t st);
+}  // namespace scope
+
+using namespace scope;
+
+static thread_local std::string g_err;
+
+static scope_status fail(scope_status s, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+extern "C" const char *scope_last_error(void) { return g_err.c_str(); }
+extern "C" int scope_version(void) { return 1; }
+
+static std::atomic<long long> g_launches{0};
+void scope::count_launches(int n) { g_launches += n; }
+extern "C" int64_t scope_kernel_launches(void) { return g_launches.load(); }
+
+// ---------------------------------------------------------------- workspace layout
+namespace {
+
+struct Layout {
+    int64_t B, H, N, D, BH;
+    int Cq, C[3], ds[3], off[3], Csum, P, Pcap, nblk, max_tiles, maxL, maxP;
+    bool f32, bisect;
+    int64_t cap;
+    size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
+    size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
+    size_t lut, item_hist, item_id, item_cnt, item_n, r, n, kh, offsets, indices, tiles, ntiles, vb;
+    size_t total;
+};
+
+size_t take(size_t &cur, size_t bytes)
+{
+    const size_t at = cur;
+    cur += (bytes + 255) & ~(size_t)255;
+    return at;
+}
+
+bool tensor_ok(const scope_tensor *t, const char *name, scope_status *st)
+{
+    if (!t) {
+        *st = fail(SCOPE_EINVAL, "%s: null tensor", name);
+        return false;
+    }
+    if (!t->ptr) {
+        *st = fail(SCOPE_EINVAL, "%s: null data pointer", name);
+        return false;
+    }
+    if (((uintptr_t)t->ptr) & 15) {
+        *st = fail(SCOPE_EALIGN, "%s: pointer not 16-byte aligned", name);
+        return false;
+    }
+    if (t->B < 1 || t->H < 1 || t->N < 1) {
+        *st = fail(SCOPE_ESHAPE, "%s: B, H, N must be >= 1 (got %lld, %lld, %lld)", name, (long long)t->B,
+                   (long long)t->H, (long long)t->N);
+        return false;
+    }
+    if (t->D != 64 && t->D != 128) {
+        *st = fail(SCOPE_ESHAPE, "%s: head dim must be 64 or 128 (got %lld)", name, (long long)t->D);
+        return false;
+    }
+    if (t->N > (1 << 24)) {
+        *st = fail(SCOPE_ESHAPE, "%s: N must be <= 2^24 (got %lld)", name, (long long)t->N);
+        return false;
+    }
+    if (t->dtype != SCOPE_F32 && t->dtype != SCOPE_BF16) {
+        *st = fail(SCOPE_EDTYPE, "%s: dtype must be f32 or bf16", name);
+        return false;
+    }
+    return true;
+}
+
+bool same_shape(const scope_tensor *a, const scope_tensor *b)
+{
+    return a->B == b->B && a->H == b->H && a->N == b->N && a->D == b->D;
+}
+
+scope_status check_params(const scope_tensor *q, const scope_grid *g, const scope_params *p)
+{
+    if (!p) return fail(SCOPE_EINVAL, "params: null");
+    const int64_t N = q->N, D = q->D;
+    const int ds[3] = {p->d_t, p->d_h, p->d_w};
+    const int C[3] = {p->c_t, p->c_h, p->c_w};
+    for (int s = 0; s < 3; ++s)
+        if (ds[s] < 0 || (ds[s] & 1)) return fail(SCOPE_ESHAPE, "params: d_t/d_h/d_w must be even and >= 0");
+    if ((int64_t)ds[0] + ds[1] + ds[2] != D) return fail(SCOPE_ESHAPE, "params: d_t + d_h + d_w must equal D");
+    if (!(p->top_p > 0.0f && p->top_p <= 1.0f)) return fail(SCOPE_EINVAL, "params: top_p must be in (0, 1]");
+    if (p->k_min < 0) return fail(SCOPE_EINVAL, "params: k_min must be >= 0");
+    if (p->iters < 0 || p->iters > 1000) return fail(SCOPE_EINVAL, "params: iters must be in [0, 1000]");
+    if (p->online_topk != 0 && p->online_topk != 1) return fail(SCOPE_EINVAL, "params: online_topk must be 0 or 1");
+    if (!(p->theta > 0.0)) return fail(SCOPE_EINVAL, "params: theta must be > 0");
+    const bool has_grid = g && (g->T != 0 || g->Hh != 0 || g->W != 0);
+    if (has_grid) {
+        if (g->T < 1 || g->Hh < 1 || g->W < 1) return fail(SCOPE_ESHAPE, "grid: T, Hh, W must all be >= 1 or all 0");
+        if ((int64_t)g->T * g->Hh * g->W != N) return fail(SCOPE_ESHAPE, "grid: T*Hh*W must equal N");
+    }
+    if (p->fixed_cluster_size < 0) return fail(SCOPE_EINVAL, "params: fixed_cluster_size must be >= 0");
+    if (p->fixed_cluster_size > 0) {
+        const int64_t f = p->fixed_cluster_size;
+        if (has_grid) return fail(SCOPE_EINVAL, "fixed_cluster_size needs grid {0,0,0} (no RoPE)");
+        if (ds[0] != D) return fail(SCOPE_ESHAPE, "fixed_cluster_size needs d_t == D, d_h == d_w == 0");
+        if (N % f) return fail(SCOPE_ESHAPE, "fixed_cluster_size must divide N");
+        int64_t m = N / f;
+        while (m > 1 && !(m & 1)) m >>= 1;
+        if (m != 1) return fail(SCOPE_ESHAPE, "N / fixed_cluster_size must be a power of two");
+        const int64_t Cn = N / f;
+        if (Cn > kMaxClusters) return fail(SCOPE_EINVAL, "N / fixed_cluster_size must be <= %d", kMaxClusters);
+        if ((p->c_q != 0 && p->c_q != Cn) || (p->c_t != 0 && p->c_t != Cn))
+            return fail(SCOPE_EINVAL, "c_q and c_t must be 0 or N / fixed_cluster_size");
+        return SCOPE_OK;
+    }
+    if (p->c_q < 1 || p->c_q > N || p->c_q > kMaxClusters)
+        return fail(SCOPE_EINVAL, "params: c_q must be in [1, min(N, %d)]", kMaxClusters);
+    int64_t P = 1;
+    for (int s = 0; s < 3; ++s) {
+        if (C[s] < 1 || C[s] > N || C[s] > kMaxClusters)
+            return fail(SCOPE_EINVAL, "params: c_t/c_h/c_w must be in [1, min(N, %d)]", kMaxClusters);
+        if (ds[s] == 0 && C[s] != 1) return fail(SCOPE_EINVAL, "params: a 0-wide subspace needs 1 cluster");
+        P *= C[s];
+    }
+    if (P > kMaxItems) return fail(SCOPE_EINVAL, "params: c_t*c_h*c_w must be <= %d", kMaxItems);
+    return SCOPE_OK;
+}
+
+Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_params *p)
+{
+    Layout L{};
+    L.B = q->B; L.H = q->H; L.N = q->N; L.D = q->D; L.BH = L.B * L.H;
+    L.f32 = q->dtype == SCOPE_F32;
+    L.bisect = p->fixed_cluster_size > 0;
+    const int ds[3] = {p->d_t, p->d_h, p->d_w};
+    if (L.bisect) {
+        const int Cn = (int)(L.N / p->fixed_cluster_size);
+        L.Cq = Cn;
+        L.C[0] = Cn; L.C[1] = 1; L.C[2] = 1;
+    } else {
+        L.Cq = p->c_q;
+        L.C[0] = p->c_t; L.C[1] = p->c_h; L.C[2] = p->c_w;
+    }
+    for (int s = 0; s < 3; ++s) L.ds[s] = ds[s];
+    L.off[0] = 0; L.off[1] = ds[0]; L.off[2] = ds[0] + ds[1];
+    L.Csum = L.C[0] + L.C[1] + L.C[2];
+    L.P = L.C[0] * L.C[1] * L.C[2];
+    L.Pcap = (int)(L.P < L.N ? L.P : L.N);
+    L.nblk = (int)((L.N + kSortBlk - 1) / kSortBlk);
+    L.max_tiles = (int)((L.N + kTQ - 1) / kTQ) + L.Cq;
+    const int T = g ? g->T : 0, Hh = g ? g->Hh : 0, W = g ? g->W : 0;
+    L.maxL = T > Hh ? T : Hh;
+    L.maxL = L.maxL > W ? L.maxL : W;
+    if (L.maxL < 1) L.maxL = 1;
+    L.maxP = 1;
+    for (int s = 0; s < 3; ++s) L.maxP = ds[s] / 2 > L.maxP ? ds[s] / 2 : L.maxP;
+    L.cap = L.BH * L.Cq * L.N;
+    const int64_t BH = L.BH, N = L.N, D = L.D;
+    size_t cur = 0;
+    L.qr = take(cur, BH * N * D * 2);
+    L.kr = take(cur, BH * N * D * 2);
+    L.qnorm = take(cur, BH * N * 4);
+    L.tab = take(cur, (size_t)3 * L.maxL * L.maxP * 16);
+    L.stats = take(cur, 64);
+    L.q_lab = take(cur, BH * N * 4);
+    L.q_cent = take(cur, BH * L.Cq * D * 4);
+    L.q_cn = take(cur, BH * L.Cq * 4);
+    L.q_sizes = take(cur, BH * L.Cq * 4);
+    L.q_perm = take(cur, BH * N * 4);
+    L.q_start = take(cur, BH * (L.Cq + 1) * 4);
+    L.q_bhist = take(cur, BH * L.Cq * L.nblk * 4);
+    L.k_codes = take(cur, 3 * BH * N * 4);
+    for (int s = 0; s < 3; ++s) {
+        L.k_cent[s] = take(cur, BH * L.C[s] * (ds[s] > 0 ? ds[s] : 1) * 4);
+        L.k_cn[s] = take(cur, BH * L.C[s] * 4);
+        L.k_sizes[s] = take(cur, BH * L.C[s] * 4);
+        L.k_perm[s] = take(cur, BH * N * 4);
+        L.k_start[s] = take(cur, BH * (L.C[s] + 1) * 4);
+        L.k_bhist[s] = take(cur, BH * L.C[s] * L.nblk * 4);
+    }
+    L.lut = take(cur, BH * L.Cq * L.Csum * 4);
+    L.item_hist = take(cur, BH * L.P * 4);
+    L.item_id = take(cur, BH * L.Pcap * 4);
+    L.item_cnt = take(cur, BH * L.Pcap * 4);
+    L.item_n = take(cur, BH * 4);
+    L.r = take(cur, BH * L.Cq * 4);
+    L.n = take(cur, BH * L.Cq * 4);
+    L.kh = take(cur, BH * 4);
+    L.offsets = take(cur, (BH * L.Cq + 1) * 8);
+    L.tiles = take(cur, BH * L.max_tiles * 8);
+    L.ntiles = take(cur, BH * 4);
+    L.vb = take(cur, L.f32 ? BH * N * D * 2 : 0);
+    L.indices = take(cur, (size_t)L.cap * 4);
+    L.total = cur;
+    return L;
+}
+
+scope_status check_device(cudaStream_t)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(SCOPE_EDEVICE, "no CUDA device");
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major != 10) return fail(SCOPE_EDEVICE, "libscope.so is built for sm_100a; device has compute capability %d.x", major);
+    static bool configured[64] = {false};
+    if (dev < 64 && !configured[dev]) {
+        if (km_configure() != cudaSuccess) return fail(SCOPE_ECUDA, "kernel attribute setup failed");
+        configured[dev] = true;
+    }
+    return SCOPE_OK;
+}
+
+scope_status launch_status(const char *what)
+{
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(SCOPE_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+    return SCOPE_OK;
+}
+
+}  // namespace
+
+struct scope_plan_s {
+    Layout L;
+    char *ws;
+    size_t ws_bytes;
+    const void *q_ptr, *k_ptr;
+    scope_dtype dtype;
+    scope_params p;
+    scope_grid g;
+};
+
+template <typename T>
+static T *at(char *ws, size_t off)
+{
+    return reinterpret_cast<T *>(ws + off);
+}
+
+extern "C" size_t scope_plan_workspace_bytes(const scope_tensor *q, const scope_grid *grid,
+                                             const scope_params *p)
+{
+    scope_status st;
+    if (!tensor_ok(q, "q", &st)) return 0;
+    if (check_params(q, grid, p) != SCOPE_OK) return 0;
+    return make_layout(q, grid, p).total;
+}
+
+static void rope_both(const Layout &L, char *ws, const scope_tensor *q, const scope_tensor *k, const scope_grid *g,
+                      const scope_params *p, cudaStream_t st)
+{
+    const bool rope = g && g->T > 0;
+    uint32_t *stats = at<uint32_t>(ws, L.stats);
+    cudaMemsetAsync(stats, 0, 64, st);
+    if (rope)
+        launch_rope_table(at<double2>(ws, L.tab), g->T, g->Hh, g->W, p->d_t, p->d_h, p->d_w, p->theta, L.maxL, L.maxP,
+                          st);
+    const int Hh = rope ? g->Hh : 1, W = rope ? g->W : 1;
+    launch_rope_apply(q->ptr, L.f32, at<__nv_bfloat16>(ws, L.qr), at<float>(ws, L.qnorm), stats + 0,
+                      at<double2>(ws, L.tab), L.BH * L.N, (int)L.N, (int)L.D, Hh, W, p->d_t, p->d_h, L.maxL, L.maxP,
+                      rope ? 1 : 0, st);
+    launch_rope_apply(k->ptr, L.f32, at<__nv_bfloat16>(ws, L.kr), nullptr, stats + 1, at<double2>(ws, L.tab),
+                      L.BH * L.N, (int)L.N, (int)L.D, Hh, W, p->d_t, p->d_h, L.maxL, L.maxP, rope ? 1 : 0, st);
+}
+
+static KmProblem key_problem(const Layout &L, char *ws, int s)
+{
+    KmProblem P{};
+    P.X = at<__nv_bfloat16>(ws, L.kr);
+    P.maxabs = at<uint32_t>(ws, L.stats) + 1;
+    P.dim_off = L.off[s];
+    P.dim_n = L.ds[s];
+    P.C = L.C[s];
+    P.labels = at<int32_t>(ws, L.k_codes) + (int64_t)s * L.BH * L.N;
+    P.cent = at<float>(ws, L.k_cent[s]);
+    P.cn = at<float>(ws, L.k_cn[s]);
+    P.sizes = at<int32_t>(ws, L.k_sizes[s]);
+    P.perm = at<int32_t>(ws, L.k_perm[s]);
+    P.start = at<int32_t>(ws, L.k_start[s]);
+    P.blockhist = at<int32_t>(ws, L.k_bhist[s]);
+    return P;
+}
+
+static KmProblem query_problem(const Layout &L, char *ws)
+{
+    KmProblem P{};
+    P.X = at<__nv_bfloat16>(ws, L.qr);
+    P.maxabs = at<uint32_t>(ws, L.stats);
+    P.dim_off = 0;
+    P.dim_n = (int)L.D;
+    P.C = L.Cq;
+    P.labels = at<int32_t>(ws, L.q_lab);
+    P.cent = at<float>(ws, L.q_cent);
+    P.cn = at<float>(ws, L.q_cn);
+    P.sizes = at<int32_t>(ws, L.q_sizes);
+    P.perm = at<int32_t>(ws, L.q_perm);
+    P.start = at<int32_t>(ws, L.q_start);
+    P.blockhist = at<int32_t>(ws, L.q_bhist);
+    return P;
+}
+
+extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k, const scope_grid *grid,
+                                   const scope_params *p, void *workspace, size_t ws_bytes, void *stream,
+                                   scope_plan_t **out)
+{
+    scope_status st;
+    if (!out) return fail(SCOPE_EINVAL, "out: null");
+    *out = nullptr;
+    if (!tensor_ok(q, "q", &st) || !tensor_ok(k, "k", &st)) return st;
+    if (!same_shape(q, k)) return fail(SCOPE_ESHAPE, "q and k shapes differ");
+    if (q->dtype != k->dtype) return fail(SCOPE_EDTYPE, "q and k dtypes differ");
+    if ((st = check_params(q, grid, p)) != SCOPE_OK) return st;
+    const Layout L = make_layout(q, grid, p);
+    if (!workspace) return fail(SCOPE_EWORKSPACE, "workspace: null");
+    if (((uintptr_t)workspace) & 255) return fail(SCOPE_EALIGN, "workspace must be 256-byte aligned");
+    if (ws_bytes < L.total)
+        return fail(SCOPE_EWORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, L.total);
+    if (L.bisect) return fail(SCOPE_EINVAL, "fixed_cluster_size: bisection path not built in this library version");
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((st = check_device(s)) != SCOPE_OK) return st;
+    char *ws = (char *)workspace;
+    const int BH = (int)L.BH, N = (int)L.N, D = (int)L.D;
+
+    rope_both(L, ws, q, k, grid, p, s);
+
+    KmBatch all{};
+    for (int i = 0; i < 3; ++i) all.p[i] = key_problem(L, ws, i);
+    all.p[3] = query_problem(L, ws);
+    all.count = 4;
+    KmBatch qonly{};
+    qonly.p[0] = all.p[3];
+    qonly.count = 1;
+    launch_km_init(all, BH, N, D, p->init_seed, s);
+    for (int it = 0; it < p->iters; ++it) {
+        launch_km_assign_direct(all, BH, N, D, s);
+        launch_km_sort(all, BH, N, s);
+        launch_km_reduce(all, BH, N, D, s);
+    }
+    launch_km_assign_direct(all, BH, N, D, s);
+    launch_km_sort(qonly, BH, N, s);
+    if ((st = launch_status("k-means")) != SCOPE_OK) return st;
+
+    launch_lut(at<float>(ws, L.q_cent), at<float>(ws, L.k_cent[0]), at<float>(ws, L.k_cent[1]),
+               at<float>(ws, L.k_cent[2]), at<float>(ws, L.lut), BH, L.Cq, D, L.ds[0], L.ds[1], L.ds[2], L.C[0],
+               L.C[1], L.C[2], s);
+    launch_items(at<int32_t>(ws, L.k_codes), at<int32_t>(ws, L.item_hist), at<int32_t>(ws, L.item_id),
+                 at<int32_t>(ws, L.item_cnt), at<int32_t>(ws, L.item_n), BH, N, L.C[1], L.C[2], L.P, L.Pcap, s);
+    run_selection(at<float>(ws, L.lut), at<int32_t>(ws, L.k_codes), at<int32_t>(ws, L.item_id),
+                  at<int32_t>(ws, L.item_cnt), at<int32_t>(ws, L.item_n), L.Pcap, N, L.Cq, L.C[0], L.C[1], L.C[2],
+                  BH, p->top_p, 1.0f / sqrtf((float)D), p->k_min, at<int32_t>(ws, L.stats) + 4,
+                  at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.r), at<int32_t>(ws, L.n), at<int32_t>(ws, L.kh),
+                  at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, s);
+    launch_tiles(at<int32_t>(ws, L.q_sizes), at<int2>(ws, L.tiles), at<int32_t>(ws, L.ntiles), BH, L.Cq, L.max_tiles,
+                 s);
+    if ((st = launch_status("selection")) != SCOPE_OK) return st;
+
+    scope_plan_s *h = (scope_plan_s *)malloc(sizeof(scope_plan_s));
+    if (!h) return fail(SCOPE_EINVAL, "host allocation of the plan handle failed");
+    h->L = L;
+    h->ws = ws;
+    h->ws_bytes = ws_bytes;
+    h->q_ptr = q->ptr;
+    h->k_ptr = k->ptr;
+    h->dtype = q->dtype;
+    h->p = *p;
+    h->g = grid ? *grid : scope_grid{0, 0, 0};
+    *out = h;
+    return SCOPE_OK;
+}
+
+static scope_status check_vo(const scope_tensor *q, const scope_tensor *v, const scope_tensor *o)
+{
+    scope_status st;
+    if (!tensor_ok(v, "v", &st) || !tensor_ok(o, "o", &st)) return st;
+    if (!same_shape(q, v) || !same_shape(q, o)) return fail(SCOPE_ESHAPE, "v and o must have q's shape");
+    if (o->dtype != SCOPE_BF16) return fail(SCOPE_EDTYPE, "o must be bf16");
+    return SCOPE_OK;
+}
+
+static const __nv_bfloat16 *v_bf16(const Layout &L, char *ws, const scope_tensor *v, cudaStream_t s)
+{
+    if (v->dtype == SCOPE_BF16) return (const __nv_bfloat16 *)v->ptr;
+    __nv_bfloat16 *vb = at<__nv_bfloat16>(ws, L.vb);
+    launch_to_bf16((const float *)v->ptr, vb, L.BH * L.N * L.D, s);
+    return vb;
+}
+
+extern "C" scope_status scope_attn(const scope_tensor *q, const scope_tensor *k, const scope_tensor *v,
+                                   const scope_plan_t *plan, scope_tensor *o, void *stream)
+{
+    scope_status st;
+    if (!plan) return fail(SCOPE_EINVAL, "plan: null");
+    if (!tensor_ok(q, "q", &st) || !tensor_ok(k, "k", &st)) return st;
+    const Layout &L = plan->L;
+    if (q->ptr != plan->q_ptr || k->ptr != plan->k_ptr)
+        return fail(SCOPE_EINVAL, "q and k must be the tensors the plan was made from");
+    if (q->B != L.B || q->H != L.H || q->N != L.N || q->D != L.D || !same_shape(q, k))
+        return fail(SCOPE_ESHAPE, "q/k shape differs from the plan's");
+    if ((st = check_vo(q, v, o)) != SCOPE_OK) return st;
+    if (v->dtype == SCOPE_F32 && !L.f32) return fail(SCOPE_EDTYPE, "f32 v needs a plan made from f32 q/k");
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((st = check_device(s)) != SCOPE_OK) return st;
+    char *ws = plan->ws;
+    const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
+    launch_attn_simt(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
+                     at<int2>(ws, L.tiles), at<int32_t>(ws, L.ntiles), L.max_tiles, at<int32_t>(ws, L.q_perm),
+                     at<int32_t>(ws, L.q_start), at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices),
+                     at<int32_t>(ws, L.n), (int)L.BH, (int)L.N, (int)L.D, L.Cq, s);
+    return launch_status("scope_attn");
+}
+
+// ---------------------------------------------------------------- dense baseline
+static Layout dense_layout(const scope_tensor *q, const scope_grid *g, const scope_params *p)
+{
+    Layout L{};
+    L.B = q->B; L.H = q->H; L.N = q->N; L.D = q->D; L.BH = L.B * L.H;
+    L.f32 = q->dtype == SCOPE_F32;
+    const int T = g ? g->T : 0, Hh = g ? g->Hh : 0, W = g ? g->W : 0;
+    L.maxL = T > Hh ? T : Hh;
+    L.maxL = L.maxL > W ? L.maxL : W;
+    if (L.maxL < 1) L.maxL = 1;
+    L.maxP = 1;
+    const int ds[3] = {p ? p->d_t : 0, p ? p->d_h : 0, p ? p->d_w : 0};
+    for (int s = 0; s < 3; ++s) L.maxP = ds[s] / 2 > L.maxP ? ds[s] / 2 : L.maxP;
+    size_t cur = 0;
+    L.qr = take(cur, L.BH * L.N * L.D * 2);
+    L.kr = take(cur, L.BH * L.N * L.D * 2);
+    L.qnorm = take(cur, L.BH * L.N * 4);
+    L.tab = take(cur, (size_t)3 * L.maxL * L.maxP * 16);
+    L.stats = take(cur, 64);
+    L.vb = take(cur, L.f32 ? L.BH * L.N * L.D * 2 : 0);
+    L.total = cur;
+    return L;
+}
+
+extern "C" size_t scope_dense_workspace_bytes(const scope_tensor *q, const scope_grid *grid,
+                                              const scope_params *p)
+{
+    scope_status st;
+    if (!tensor_ok(q, "q", &st)) return 0;
+    if (!p) {
+        fail(SCOPE_EINVAL, "params: null");
+        return 0;
+    }
+    const bool has_grid = grid && (grid->T || grid->Hh || grid->W);
+    return dense_layout(q, has_grid ? grid : nullptr, p).total;
+}
+
+extern "C" scope_status scope_dense_attn(const scope_tensor *q, const scope_tensor *k, const scope_tensor *v,
+                                         const scope_grid *grid, const scope_params *p, scope_tensor *o,
+                                         void *workspace, size_t ws_bytes, void *stream)
+{
+    scope_status st;
+    if (!tensor_ok(q, "q", &st) || !tensor_ok(k, "k", &st)) return st;
+    if (!same_shape(q, k)) return fail(SCOPE_ESHAPE, "q and k shapes differ");
+    if (q->dtype != k->dtype) return fail(SCOPE_EDTYPE, "q and k dtypes differ");
+    if ((st = check_vo(q, v, o)) != SCOPE_OK) return st;
+    if (v->dtype != q->dtype) return fail(SCOPE_EDTYPE, "v dtype must match q");
+    if (!p) return fail(SCOPE_EINVAL, "params: null");
+    const bool has_grid = grid && (grid->T || grid->Hh || grid->W);
+    if (has_grid) {
+        if (grid->T < 1 || grid->Hh < 1 || grid->W < 1 || (int64_t)grid->T * grid->Hh * grid->W != q->N)
+            return fail(SCOPE_ESHAPE, "grid: T*Hh*W must equal N");
+        if (p->d_t < 0 || p->d_h < 0 || p->d_w < 0 || (p->d_t | p->d_h | p->d_w) & 1 ||
+            (int64_t)p->d_t + p->d_h + p->d_w != q->D)
+            return fail(SCOPE_ESHAPE, "params: d_t/d_h/d_w must be even and sum to D");
+        if (!(p->theta > 0.0)) return fail(SCOPE_EINVAL, "params: theta must be > 0");
+    }
+    const Layout L = dense_layout(q, has_grid ? grid : nullptr, p);
+    if (!workspace) return fail(SCOPE_EWORKSPACE, "workspace: null");
+    if (((uintptr_t)workspace) & 255) return fail(SCOPE_EALIGN, "workspace must be 256-byte aligned");
+    if (ws_bytes < L.total) return fail(SCOPE_EWORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, L.total);
+    cudaStream_t s = (cudaStream_t)stream;
+    if ((st = check_device(s)) != SCOPE_OK) return st;
+    char *ws = (char *)workspace;
+    rope_both(L, ws, q, k, has_grid ? grid : nullptr, p, s);
+    const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
+    launch_attn_simt(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr, nullptr,
+                     nullptr, 0, nullptr, nullptr, nullptr, nullptr, nullptr, (int)L.BH, (int)L.N, (int)L.D, 1, s);
+    return launch_status("scope_dense_attn");
+}
+
+// ---------------------------------------------------------------- views / status
+extern "C" scope_status scope_plan_view(const scope_plan_t *plan, int which, scope_view *out)
+{
+    if (!plan || !out) return fail(SCOPE_EINVAL, "plan/out: null");
+    const Layout &L = plan->L;
+    char *ws = plan->ws;
+    const int64_t B = L.B, H = L.H, N = L.N, D = L.D;
+    scope_view v{};
+    auto set = [&](size_t off, scope_dtype dt, int nd, int64_t a, int64_t b, int64_t c, int64_t d) {
+        v.ptr = ws + off;
+        v.dtype = dt;
+        v.ndim = nd;
+        v.shape[0] = a; v.shape[1] = b; v.shape[2] = c; v.shape[3] = d;
+    };
+    switch (which) {
+    case SCOPE_VIEW_QR: set(L.qr, SCOPE_BF16, 4, B, H, N, D); break;
+    case SCOPE_VIEW_KR: set(L.kr, SCOPE_BF16, 4, B, H, N, D); break;
+    case SCOPE_VIEW_Q_LABELS: set(L.q_lab, SCOPE_I32, 3, B, H, N, 0); break;
+    case SCOPE_VIEW_Q_CENTROIDS: set(L.q_cent, SCOPE_F32, 4, B, H, L.Cq, D); break;
+    case SCOPE_VIEW_Q_SIZES: set(L.q_sizes, SCOPE_I32, 3, B, H, L.Cq, 0); break;
+    case SCOPE_VIEW_Q_PERM: set(L.q_perm, SCOPE_I32, 3, B, H, N, 0); break;
+    case SCOPE_VIEW_Q_START: set(L.q_start, SCOPE_I32, 3, B, H, L.Cq + 1, 0); break;
+    case SCOPE_VIEW_K_CODES: set(L.k_codes, SCOPE_I32, 4, 3, B, H, N); break;
+    case SCOPE_VIEW_K_CENT_T: set(L.k_cent[0], SCOPE_F32, 4, B, H, L.C[0], L.ds[0]); break;
+    case SCOPE_VIEW_K_CENT_H: set(L.k_cent[1], SCOPE_F32, 4, B, H, L.C[1], L.ds[1]); break;
+    case SCOPE_VIEW_K_CENT_W: set(L.k_cent[2], SCOPE_F32, 4, B, H, L.C[2], L.ds[2]); break;
+    case SCOPE_VIEW_LUT: set(L.lut, SCOPE_F32, 4, B, H, L.Cq, L.Csum); break;
+    case SCOPE_VIEW_R: set(L.r, SCOPE_I32, 3, B, H, L.Cq, 0); break;
+    case SCOPE_VIEW_KH: set(L.kh, SCOPE_I32, 2, B, H, 0, 0); break;
+    case SCOPE_VIEW_N: set(L.n, SCOPE_I32, 3, B, H, L.Cq, 0); break;
+    case SCOPE_VIEW_OFFSETS: set(L.offsets, SCOPE_I64, 1, L.BH * L.Cq + 1, 0, 0, 0); break;
+    case SCOPE_VIEW_INDICES: set(L.indices, SCOPE_I32, 1, L.cap, 0, 0, 0); break;
+    case SCOPE_VIEW_ERROR: set(L.stats + 16, SCOPE_I32, 1, 4, 0, 0, 0); break;
+    default: return fail(SCOPE_EINVAL, "view id %d out of range", which);
+    }
+    *out = v;
+    return SCOPE_OK;
+}
+
+extern "C" scope_status scope_sync_status(const scope_plan_t *plan, void *stream)
+{
+    if (!plan) return fail(SCOPE_EINVAL, "plan: null");
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(SCOPE_ECUDA, "stream: %s", cudaGetErrorString(e));
+    int32_t err[4] = {0, 0, 0, 0};
+    e = cudaMemcpy(err, plan->ws + plan->L.stats + 16, sizeof err, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(SCOPE_ECUDA, "reading the error word: %s", cudaGetErrorString(e));
+    if (err[0] & kErrTimeout) return fail(SCOPE_ETIMEOUT, "a bounded device wait gave up (detail 0x%x)", err[1]);
+    if (err[0]) return fail(SCOPE_EDEVICE, "device range check fired (flags 0x%x, detail 0x%x)", err[0], err[1]);
+    return SCOPE_OK;
+}
+
+extern "C" void scope_plan_destroy(scope_plan_t *plan) { free(plan); }

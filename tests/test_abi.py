@@ -1,0 +1,130 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol
+include/scope.h declares, and rejects bad arguments before any device work.
+
+The pointers used here are fake, 16-byte aligned addresses: every call below
+must fail in argument validation, which runs before any CUDA call."""
+import ctypes
+
+import pytest
+
+import cluster_guided_sparse_b200 as scope
+from cluster_guided_sparse_b200 import build, synth
+
+FAKE = 0x7F0000000000  # aligned, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return scope.lib()
+
+
+def T(N=256, D=64, dtype=scope.SCOPE_BF16, ptr=FAKE, B=1, H=2):
+    return scope.ScopeTensor(ptr, dtype, B, H, N, D)
+
+
+def P(**kw):
+    return scope.make_params(synth.WORKLOADS["tiny"], **kw)
+
+
+def plan_status(L, q, k, params, grid, ws=FAKE, ws_bytes=1 << 40):
+    h = ctypes.c_void_p()
+    st = L.scope_plan(ctypes.byref(q), ctypes.byref(k), ctypes.byref(grid), ctypes.byref(params),
+                      ctypes.c_void_p(ws), ws_bytes, None, ctypes.byref(h))
+    return st, L.scope_last_error().decode()
+
+
+def test_exports_every_declared_symbol(L):
+    names = scope.header_symbols()
+    assert "scope_plan" in names and "scope_attn" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.scope_version() >= 1
+
+
+def test_workspace_bytes_counts_list_capacity(L):
+    p, g = P()
+    q = T()
+    n = L.scope_plan_workspace_bytes(ctypes.byref(q), ctypes.byref(g), ctypes.byref(p))
+    # worst-case lists (c_q * N per head), post-RoPE copies, and more
+    assert n >= 2 * 8 * 256 * 4 + 2 * 2 * 256 * 64 * 2
+    q2 = T(H=4)
+    assert L.scope_plan_workspace_bytes(ctypes.byref(q2), ctypes.byref(g), ctypes.byref(p)) > n
+
+
+@pytest.mark.parametrize("mut,code,msg", [
+    (dict(top_p=0.0), 1, "top_p"),
+    (dict(top_p=1.5), 1, "top_p"),
+    (dict(k_min=-1), 1, "k_min"),
+    (dict(d_t=15, d_h=25), 2, "even"),
+    (dict(d_t=16, d_h=24, d_w=26), 2, "equal D"),
+    (dict(c_q=0), 1, "c_q"),
+    (dict(c_q=257), 1, "c_q"),
+    (dict(c_t=300), 1, "c_t"),
+    (dict(grid=(4, 8, 7)), 2, "grid"),
+    (dict(grid=(4, 0, 64)), 2, "grid"),
+    (dict(iters=-1), 1, "iters"),
+    (dict(online_topk=2), 1, "online_topk"),
+    (dict(fixed_cluster_size=64), 1, "grid"),
+])
+def test_bad_params_rejected_on_host(L, mut, code, msg):
+    p, g = P(**mut)
+    st, err = plan_status(L, T(), T(), p, g)
+    assert st == code and msg in err, (st, err)
+    assert L.scope_plan_workspace_bytes(ctypes.byref(T()), ctypes.byref(g), ctypes.byref(p)) == 0
+
+
+def test_bad_tensors_rejected_on_host(L):
+    p, g = P()
+    assert plan_status(L, T(ptr=FAKE + 8), T(), p, g)[0] == 4  # misaligned
+    assert plan_status(L, T(ptr=0), T(), p, g)[0] == 1  # null
+    assert plan_status(L, T(D=96), T(D=96), p, g)[0] == 2  # head dim
+    assert plan_status(L, T(), T(N=128), p, g)[0] == 2  # shape mismatch
+    assert plan_status(L, T(), T(dtype=scope.SCOPE_F32), p, g)[0] == 3  # dtype mismatch
+    assert plan_status(L, T(dtype=7), T(dtype=7), p, g)[0] == 3
+
+
+def test_workspace_checks_on_host(L):
+    p, g = P()
+    assert plan_status(L, T(), T(), p, g, ws=0)[0] == 5
+    assert plan_status(L, T(), T(), p, g, ws=FAKE + 16)[0] == 4
+    st, err = plan_status(L, T(), T(), p, g, ws_bytes=1024)
+    assert st == 5 and "too small" in err
+
+
+def test_fixed_cluster_size_shape_rules(L):
+    q = T(N=65536 - 64, D=64)  # 1023 clusters of 64: not a power of two
+    p, g = scope.make_params(synth.WORKLOADS["unstructured"])
+    assert plan_status(L, q, q, p, g)[0] == 2
+    p2, g2 = scope.make_params(synth.WORKLOADS["unstructured"], d_t=32, d_h=32)
+    assert plan_status(L, T(N=65536), T(N=65536), p2, g2)[0] == 2
+
+
+def test_attn_and_views_reject_null_plan(L):
+    q = T()
+    assert L.scope_attn(ctypes.byref(q), ctypes.byref(q), ctypes.byref(q), None, ctypes.byref(q), None) == 1
+    v = scope.ScopeView()
+    assert L.scope_plan_view(None, 0, ctypes.byref(v)) == 1
+    assert L.scope_sync_status(None, None) == 1
+    L.scope_plan_destroy(None)  # freeing a null handle is a no-op
+
+
+def test_dense_rejects_bad_grid(L):
+    p, g = P(grid=(4, 8, 9))
+    q = T()
+    o = T()
+    st = L.scope_dense_attn(ctypes.byref(q), ctypes.byref(q), ctypes.byref(q), ctypes.byref(g), ctypes.byref(p),
+                            ctypes.byref(o), ctypes.c_void_p(FAKE), 1 << 40, None)
+    assert st == 2
+    f = T(dtype=scope.SCOPE_F32)
+    p, g = P()
+    st = L.scope_dense_attn(ctypes.byref(q), ctypes.byref(q), ctypes.byref(q), ctypes.byref(g), ctypes.byref(p),
+                            ctypes.byref(f), ctypes.c_void_p(FAKE), 1 << 40, None)
+    assert st == 3  # output must be bf16
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(scope, "_lib", None)
+    monkeypatch.setattr(scope, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        scope.lib()

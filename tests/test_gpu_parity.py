@@ -1,0 +1,247 @@
+"""CUDA path vs the fp64 oracle, stage by stage, through the C ABI.
+
+Small workloads are checked in full; the Wan-480p and HunyuanVideo-720p sized
+workloads at their full sizes on sampled heads, rows, clusters and queries.
+Tolerances and the near-tie rule are in parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import cluster_guided_sparse_b200 as scope
+import oracle
+import parity as P
+from cluster_guided_sparse_b200 import synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def to_dev(*ts):
+    return [t.to(DEV).contiguous() for t in ts]
+
+
+def plan_of(w, q, k, **kw):
+    params, grid = scope.make_params(w, **kw)
+    return scope.plan(q, k, params, grid)
+
+
+def pull(pl, w, heads):
+    """Host copies of one plan's per-head results."""
+    out = {}
+    B = 0
+    lab = pl.view("q_labels")
+    cent = pl.view("q_centroids")
+    codes = pl.view("k_codes")
+    kc = [pl.view("k_cent_t"), pl.view("k_cent_h"), pl.view("k_cent_w")]
+    for h in heads:
+        out[h] = dict(
+            q_labels=lab[B, h].cpu().numpy(),
+            q_cent=P.np64(cent[B, h]),
+            codes=[codes[s, B, h].cpu().numpy() for s in range(3)],
+            k_cent=[P.np64(kc[s][B, h]) for s in range(3)],
+        )
+    return out
+
+
+def lists_fn(pl, w, h, B=0):
+    off = pl.view("offsets").cpu().numpy()
+    n = pl.view("n").cpu().numpy()
+    idx = pl.view("indices")
+
+    def get(c):
+        i = (B * w.H + h) * w.c_q + c if w.fixed_cluster_size == 0 else (B * w.H + h) * (w.N // w.fixed_cluster_size) + c
+        return idx[int(off[i]):int(off[i]) + int(n[B, h, c])].cpu().numpy()
+    return get
+
+
+def stagefed(w, heads, iters_list, row_sample=None, cl_sample=None, q_sample=None, seed=0):
+    rng = np.random.default_rng(seed)
+    q, k, v = synth.make_inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    N, D = w.N, w.D
+    rows = np.sort(rng.choice(N, row_sample, replace=False)) if row_sample else np.arange(N)
+    states = {}
+    for it in iters_list:
+        pl = plan_of(w, qd, kd, iters=it)
+        states[it] = pull(pl, w, heads)
+        if it == iters_list[-1]:
+            final = pl
+        else:
+            del pl
+    torch.cuda.synchronize()
+    final.sync_status()
+    qr_all, kr_all = final.view("qr"), final.view("kr")
+    o = scope.attn(qd, kd, vd, final)
+    torch.cuda.synchronize()
+    tc_q, tc_k, tc_sel = P.TieCounter(), P.TieCounter(), P.TieCounter()
+    offs = np.cumsum((0,) + tuple(w.d_split))
+    report = {}
+    for h in heads:
+        qr, kr = P.np64(qr_all[0, h]), P.np64(kr_all[0, h])
+        P.check_rope(qr[rows], q[0, h].double().numpy(), w, rows)
+        P.check_rope(kr[rows], k[0, h].double().numpy(), w, rows)
+        for i, it in enumerate(iters_list):
+            st = states[it][h]
+            if it == 0:  # strided init: exact rows
+                stride = N // w.c_q
+                np.testing.assert_array_equal(st["q_cent"], qr[np.arange(w.c_q) * stride])
+            P.check_assign(qr[rows], st["q_cent"], st["q_labels"][rows], tc_q, f"h{h} it{it} queries")
+            for s in range(3):
+                a, b = int(offs[s]), int(offs[s + 1])
+                P.check_assign(kr[rows, a:b], st["k_cent"][s], st["codes"][s][rows], tc_k, f"h{h} it{it} keys s{s}")
+            if i > 0 and iters_list[i - 1] == it - 1:
+                prev = states[it - 1][h]
+                P.check_update(qr, prev["q_labels"], prev["q_cent"], st["q_cent"], f"h{h} it{it} query update")
+                for s in range(3):
+                    a, b = int(offs[s]), int(offs[s + 1])
+                    P.check_update(kr[:, a:b], prev["codes"][s], prev["k_cent"][s], st["k_cent"][s],
+                                   f"h{h} it{it} key update s{s}")
+        st = states[iters_list[-1]][h]
+        lut = final.view("lut")[0, h].cpu().numpy()
+        P.check_lut(st["q_cent"], st["k_cent"], w.d_split, lut.astype(np.float64))
+        sizes = final.view("q_sizes")[0, h].cpu().numpy()
+        assert (sizes == np.bincount(st["q_labels"], minlength=w.c_q)).all()
+        perm = final.view("q_perm")[0, h].cpu().numpy()
+        qstart = final.view("q_start")[0, h].cpu().numpy()
+        assert (perm == np.argsort(st["q_labels"], kind="stable")).all()
+        assert (np.diff(qstart) == sizes).all()
+        clusters = np.arange(w.c_q) if cl_sample is None else rng.choice(w.c_q, cl_sample, replace=False)
+        get = lists_fn(final, w, h)
+        P.check_selection(lut, st["codes"], sizes, final.view("r")[0, h].cpu().numpy(),
+                          final.view("kh")[0, h].item(), final.view("n")[0, h].cpu().numpy(), get, w, N, D,
+                          clusters, tc_sel)
+        qrows = np.arange(N) if q_sample is None else np.sort(rng.choice(N, q_sample, replace=False))
+        report[h] = P.check_attention(qr, kr, v[0, h].double().numpy(), st["q_labels"], get,
+                                      P.np64(o[0, h]), qrows)
+    tc_q.assert_ok("query assign")
+    tc_k.assert_ok("key assign")
+    tc_sel.assert_ok("Top-p counts")
+    return report
+
+
+def test_tiny_config_full_parity():
+    w = synth.WORKLOADS["tiny"]
+    stagefed(w, range(w.H), list(range(w.iters + 1)))
+
+
+def test_small_config_full_parity():
+    w = synth.WORKLOADS["small"]
+    stagefed(w, range(w.H), list(range(w.iters + 1)))
+
+
+@pytest.mark.parametrize("top_p", [0.8, 0.9, 0.95])
+def test_wan480p_sampled_parity(top_p):
+    w = synth.WORKLOADS["wan480p"].with_(top_p=top_p)
+    iters = [0, 1, 2, 9, 10] if top_p == 0.9 else [10]
+    stagefed(w, [0, w.H // 2, w.H - 1], iters, row_sample=3000, cl_sample=6, q_sample=48)
+
+
+def test_hunyuan720p_sampled_parity():
+    w = synth.WORKLOADS["hunyuan720p"]
+    stagefed(w, [0, w.H - 1], [0, 1, 9, 10], row_sample=2000, cl_sample=4, q_sample=32)
+
+
+def test_plan_is_deterministic():
+    w = synth.WORKLOADS["small"]
+    qd, kd, _ = to_dev(*synth.make_inputs(w))
+    a, b = plan_of(w, qd, kd), plan_of(w, qd, kd)
+    torch.cuda.synchronize()
+    for name in ("q_labels", "k_codes", "q_centroids", "r", "kh", "n", "offsets"):
+        assert torch.equal(a.view(name), b.view(name)), name
+    tot = int(a.view("offsets")[-1])
+    assert torch.equal(a.view("indices")[:tot], b.view("indices")[:tot])
+
+
+@pytest.mark.parametrize("name", ["tiny", "small", "wan480p"])
+def test_dense_attention_parity(name):
+    w = synth.WORKLOADS[name]
+    q, k, v = synth.make_inputs(w, heads=[0, 1]) if w.H > 2 else synth.make_inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    params, grid = scope.make_params(w)
+    o = scope.dense_attn(qd, kd, vd, params, grid)
+    torch.cuda.synchronize()
+    rows = np.arange(w.N) if w.N <= 2048 else np.sort(np.random.default_rng(1).choice(w.N, 64, replace=False))
+    for h in range(q.shape[1]):
+        qr = oracle.rope3d(q[0, h].double().numpy(), w.grid, w.d_split, w.theta)
+        kr = oracle.rope3d(k[0, h].double().numpy(), w.grid, w.d_split, w.theta)
+        qr, kr = oracle._round_bf16(qr), oracle._round_bf16(kr)
+        ref = oracle.attention_rows(qr[rows], kr, v[0, h].double().numpy(), np.arange(w.N, dtype=np.int32),
+                                    1.0 / np.sqrt(w.D))
+        max_abs, rel = P.attn_error(P.np64(o[0, h])[rows], ref)
+        assert max_abs <= P.ATTN_MAX_ABS and rel <= P.ATTN_REL_L2, (max_abs, rel)
+
+
+def test_top_p_one_equals_dense():
+    w = synth.WORKLOADS["small"].with_(top_p=1.0)
+    qd, kd, vd = to_dev(*synth.make_inputs(w))
+    pl = plan_of(w, qd, kd)
+    o = scope.attn(qd, kd, vd, pl)
+    params, grid = scope.make_params(w)
+    od = scope.dense_attn(qd, kd, vd, params, grid)
+    torch.cuda.synchronize()
+    assert (pl.view("n") == w.N).all()
+    max_abs, rel = P.attn_error(P.np64(o), P.np64(od))
+    assert max_abs <= 1e-2 and rel <= 2e-3, (max_abs, rel)
+
+
+@pytest.mark.parametrize("case", [
+    dict(N=105, D=64, grid=(3, 5, 7), d_split=(16, 24, 24), c_q=5, c_sub=(3, 4, 5)),   # ragged everything
+    dict(N=64, D=64, grid=(1, 8, 8), d_split=(0, 32, 32), c_q=1, c_sub=(1, 8, 8)),     # one cluster, empty t block
+    dict(N=300, D=128, grid=(3, 10, 10), d_split=(16, 56, 56), c_q=7, c_sub=(4, 4, 4), top_p=1.0),
+    dict(N=200, D=64, grid=(2, 10, 10), d_split=(16, 24, 24), c_q=6, c_sub=(2, 2, 2), k_min=500),
+    dict(N=200, D=64, grid=(2, 10, 10), d_split=(16, 24, 24), c_q=6, c_sub=(3, 3, 3), online_topk=0, iters=0),
+    dict(N=256, D=64, grid=(0, 0, 0), d_split=(16, 24, 24), c_q=8, c_sub=(4, 4, 4), top_p=0.5),  # no grid
+    dict(N=512, D=128, grid=(2, 16, 16), d_split=(16, 56, 56), c_q=16, c_sub=(8, 8, 8), H=3, B=2),
+])
+def test_edge_cases(case):
+    case = dict(case)
+    B = case.pop("B", 1)
+    w, (q, k, v) = synth.tiny_case(**case)
+    if B > 1:
+        w = w.with_(B=B)
+        q, k, v = synth.make_inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    pl = plan_of(w, qd, kd)
+    o = scope.attn(qd, kd, vd, pl)
+    torch.cuda.synchronize()
+    pl.sync_status()
+    N, D = w.N, w.D
+    tc = P.TieCounter()
+    for b in range(w.B):
+        for h in range(w.H):
+            qr, kr = P.np64(pl.view("qr")[b, h]), P.np64(pl.view("kr")[b, h])
+            if w.grid[0]:
+                P.check_rope(qr, q[b, h].double().numpy(), w)
+            lab = pl.view("q_labels")[b, h].cpu().numpy()
+            cent = P.np64(pl.view("q_centroids")[b, h])
+            P.check_assign(qr, cent, lab, tc)
+            codes = [pl.view("k_codes")[s, b, h].cpu().numpy() for s in range(3)]
+            lut = pl.view("lut")[b, h].cpu().numpy()
+            sizes = pl.view("q_sizes")[b, h].cpu().numpy()
+            get = lists_fn(pl, w, h, B=b)
+            P.check_selection(lut, codes, sizes, pl.view("r")[b, h].cpu().numpy(), pl.view("kh")[b, h].item(),
+                              pl.view("n")[b, h].cpu().numpy(), get, w, N, D, range(w.c_q), tc)
+            P.check_attention(qr, kr, v[b, h].double().numpy(), lab, get, P.np64(o[b, h]), np.arange(N))
+    tc.assert_ok("edge")
+
+
+def test_degenerate_identical_tokens_leave_clusters_empty():
+    w, _ = synth.tiny_case(N=128, D=64, grid=(2, 8, 8), d_split=(16, 24, 24), c_q=4, c_sub=(2, 2, 2))
+    q = torch.ones((1, 1, 128, 64))
+    k = torch.ones((1, 1, 128, 64))
+    v = torch.randn((1, 1, 128, 64), generator=torch.Generator().manual_seed(0))
+    w = w.with_(grid=(0, 0, 0))
+    qd, kd, vd = to_dev(q, k, v)
+    pl = plan_of(w, qd, kd)
+    o = scope.attn(qd, kd, vd, pl)
+    torch.cuda.synchronize()
+    sizes = pl.view("q_sizes")[0, 0].cpu().numpy()
+    assert sizes.tolist() == [128, 0, 0, 0]  # all equal -> lowest index wins, others stay empty
+    n = pl.view("n")[0, 0].cpu().numpy()
+    assert n[1:].tolist() == [0, 0, 0]
+    # equal logits: attention is the mean of V over the selected keys
+    get = lists_fn(pl, w, 0)
+    sel = get(0)
+    np.testing.assert_allclose(P.np64(o[0, 0]), np.broadcast_to(v[0, 0].double().numpy()[sel].mean(0), (128, 64)),
+                               atol=2e-2)
