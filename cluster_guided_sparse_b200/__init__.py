@@ -214,3 +214,24 @@ def dense_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: ScopeP
                                   ctypes.byref(grid), ctypes.byref(params), ctypes.byref(as_tensor(out)),
                                   ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)))
     return out
+
+
+def kmeans_noalloc(x: torch.Tensor, dim_off: int, dim_n: int, C: int, iters: int, seed: int = 0,
+                   labels: Optional[torch.Tensor] = None, centroids: Optional[torch.Tensor] = None,
+                   stream=None):
+    """scope_kmeans_noalloc: k-means of columns [dim_off, dim_off+dim_n) of a bf16
+    [B, H, N, D] device tensor using the library's fixed scratch (no workspace).
+    Returns (labels int32 [B,H,N], centroids f32 [B,H,C,dim_n])."""
+    L = lib()
+    f = L.scope_kmeans_noalloc
+    f.argtypes = [ctypes.POINTER(ScopeTensor), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    B, H, N, _ = x.shape
+    if labels is None:
+        labels = torch.empty((B, H, N), dtype=torch.int32, device=x.device)
+    if centroids is None:
+        centroids = torch.empty((B, H, C, dim_n), dtype=torch.float32, device=x.device)
+    _check(f(ctypes.byref(as_tensor(x)), dim_off, dim_n, C, iters, seed & 0xFFFFFFFF,
+             ctypes.c_void_p(labels.data_ptr()), ctypes.c_void_p(centroids.data_ptr()), _stream(stream)))
+    return labels, centroids

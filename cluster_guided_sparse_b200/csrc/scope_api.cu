@@ -54,6 +54,9 @@ static scope_status fail(scope_status s, const char *fmt, ...)
 }
 
 extern "C" const char *scope_last_error(void) { return g_err.c_str(); }
+
+// Lets other translation units of the library report an error message.
+scope_status scope_set_error(scope_status s, const char *msg) { return fail(s, "%s", msg); }
 extern "C" int scope_version(void) { return 1; }
 
 static std::atomic<long long> g_launches{0};

@@ -191,6 +191,35 @@ const char *scope_last_error(void);
 /* Library version, for the binding's load check. */
 int scope_version(void);
 
+/* ---------------------------------------------------------------------- */
+/* Clustering without device allocation.  The pages have no counterpart of  */
+/* this entry point; it exists for callers that cannot allocate device      */
+/* memory (a plain C program without an allocator, a server whose device    */
+/* memory plan is fixed after start-up, a plug-in that may only touch the   */
+/* buffers its host passes in).                                             */
+/*                                                                          */
+/* scope_kmeans_noalloc runs the same Lloyd k-means as scope_plan's step 2  */
+/* on columns [dim_off, dim_off + dim_n) of x, with the same strided init,  */
+/* tie rule, empty-cluster rule and final assign, so its results equal the  */
+/* plan's for the same rows.                                                */
+/*   x          bf16 [B,H,N,D] device, D in {64, 128} (e.g. post-RoPE rows). */
+/*   labels     int32 [B,H,N] device, written (final assign).               */
+/*   centroids  f32 [B,H,C,dim_n] device, written (after the last update).  */
+/* Scratch: a fixed SCOPE_NOALLOC_SCRATCH_BYTES array inside the library,   */
+/* held on every GPU that loads it until the process exits.  The first call */
+/* on a device looks up that array's device address (make it before any    */
+/* stream capture).  All calls share the array: calls whose device work     */
+/* overlaps race and must be serialised by the caller.  A shape needing     */
+/* more than the array (scope_kmeans_noalloc_scratch_bytes) returns         */
+/* SCOPE_ECAPACITY before any launch.  Allocates nothing.                   */
+/* ---------------------------------------------------------------------- */
+#define SCOPE_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+size_t scope_kmeans_noalloc_scratch_bytes(int64_t B, int64_t H, int64_t N, int32_t C);
+scope_status scope_kmeans_noalloc(const scope_tensor *x, int32_t dim_off, int32_t dim_n,
+                                  int32_t C, int32_t iters, uint32_t init_seed,
+                                  int32_t *labels, float *centroids, void *stream);
+
 /* Number of kernels this library has launched in this process so far (all
  * devices, all threads); a diagnostic for launch accounting. */
 int64_t scope_kernel_launches(void);
