@@ -1,0 +1,505 @@
+// Step 5 of SCOPE (abstract: "sparse attention is then computed over the
+// selected original keys and values") on the 5th-generation tensor cores.
+//
+// One CTA = one work item = up to 256 queries of one query cluster (two
+// 128-row Q tiles) against that cluster's selected-key list, walked in tiles
+// of 128 keys.  Both Q tiles share every gathered K/V tile, which halves the
+// K/V bytes per flop (the tiles come from L2: a head's K/V is 61 MB at 720p).
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax / epilogue of Q tile 0 (one thread per query row)
+//   warps 4-7  softmax / epilogue of Q tile 1
+//   warp 8     tcgen05.mma issuer (one lane), owns the TMEM allocation
+//   warp 9     producer: gathers Q rows and the listed K/V rows with 16-byte
+//              cp.async into 128B-swizzled shared-memory tiles (2 stages)
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
+// S = Q K^T lands in TMEM (fp32); the softmax rows read it with tcgen05.ld,
+// write P as packed bf16 over the first 64 columns of their S, and the
+// issuer runs O += P V with P taken from TMEM and V from shared memory.
+// Online softmax in base 2 with a lazy rescale: O and l are rescaled only
+// when a row's max grows by more than 2^8, so P never exceeds 256.
+//
+// Every mbarrier wait is bounded (about two seconds of clock64); on timeout
+// the thread records SCOPE's timeout bit in the device error word, the CTA
+// abandons its work item, and all threads still meet at the final barrier
+// so the TMEM is released.
+#include "common.cuh"
+
+namespace scope {
+
+namespace tc {
+
+constexpr int kThreads = 320;
+constexpr int BN = 128;       // keys per K/V tile
+constexpr int BM = 128;       // rows per Q tile
+constexpr long long kWaitCycles = 4000000000ll;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: false after ~2 s or once another thread of the CTA aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *err, int where)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0u) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > kWaitCycles) {
+                *abort_flag = 1;
+                set_error(err, kErrTimeout, where);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100 version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: bf16 A/B, f32 accumulate, M=128.
+__device__ __forceinline__ uint32_t idesc_bf16(int n, bool b_mn_major)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+#define SCOPE_R32(r) \
+    "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), \
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),  \
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), \
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define SCOPE_W32(r) \
+    "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), \
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),          \
+        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]),          \
+        "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : SCOPE_R32(r)
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        SCOPE_W32(r)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Byte offset of 16-byte chunk `c` (0 .. D/8-1) of row `r` in a [rows][D] bf16
+// tile stored as D/64 column blocks of rows x 128 B, 128B-swizzled.
+__device__ __forceinline__ uint32_t sw_off(int r, int c, int rows)
+{
+    return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+struct Args {
+    const __nv_bfloat16 *qr, *kr, *v;
+    __nv_bfloat16 *o;
+    const int4 *items;         // (bh, cluster, first query, query count) per work item
+    const int32_t *n_items;    // total work items
+    const int32_t *perm;       // [BH][N] or null (dense: identity)
+    const int32_t *start;      // [BH][Cq+1] or null
+    const long long *offsets;  // [BH*Cq] or null (dense: all keys)
+    const int32_t *indices;
+    const int32_t *n_c;        // [BH][Cq] or null
+    int32_t *err;
+    int N, Cq;
+    float scale_log2;          // log2(e) / sqrt(D)
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Args a)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte alignment for the swizzle atoms.
+    unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    constexpr int QT_BYTES = BM * D * 2;
+    constexpr int KV_BYTES = BN * D * 2;
+    unsigned char *sQ = sm;                      // 2 Q tiles
+    unsigned char *sK = sm + 2 * QT_BYTES;       // 2 stages
+    unsigned char *sV = sK + 2 * KV_BYTES;       // 2 stages
+
+    __shared__ uint64_t bar_q, bar_kv_full[2], bar_kv_empty[2], bar_s_full[2], bar_p_full[2], bar_o_final[2];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int item = blockIdx.x;
+    if (item >= *a.n_items) return;  // uniform for the CTA
+    const int4 it = a.items[item];
+    const int bh = it.x, c = it.y, q0 = it.z, nq = it.w;
+    const bool two = nq > BM;
+    const int64_t base = (int64_t)bh * a.N;
+    const int cstart = a.start ? a.start[(int64_t)bh * (a.Cq + 1) + c] : 0;
+    const long long loff = a.indices ? a.offsets[(int64_t)bh * a.Cq + c] : 0;
+    const int nk = a.indices ? a.n_c[(int64_t)bh * a.Cq + c] : a.N;
+    const int ntiles = (nk + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bar_q, 32);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar_kv_full[i], 32);
+            mbar_init(&bar_kv_empty[i], 1);
+            mbar_init(&bar_s_full[i], 1);
+            mbar_init(&bar_p_full[i], 128);
+            mbar_init(&bar_o_final[i], 1);
+        }
+        abort_sh = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 8) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&tmem_base_sh)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    volatile int *abort_flag = &abort_sh;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ producer
+        // Q rows (zero-filled past the work item's queries).
+        for (int t = 0; t < 2; ++t) {
+            const uint32_t dst0 = smem_u32(sQ + t * QT_BYTES);
+            for (int r = lane; r < BM; r += 32) {
+                const int qi = t * BM + r;
+                const bool ok = qi < nq;
+                const int tok = ok ? (a.perm ? a.perm[base + cstart + q0 + qi] : q0 + qi) : 0;
+                const __nv_bfloat16 *src = a.qr + (base + tok) * D;
+#pragma unroll
+                for (int ch = 0; ch < D / 8; ++ch) cp_async16(dst0 + sw_off(r, ch, BM), src + ch * 8, ok);
+            }
+        }
+        cp_async_commit();
+        cp_async_wait_all();
+        fence_async_smem();
+        mbar_arrive(&bar_q);
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j & 1;
+            if (j >= 2 && !mbar_wait(&bar_kv_empty[s], ((j >> 1) - 1) & 1, abort_flag, a.err, 0x10)) break;
+            const uint32_t dk = smem_u32(sK + s * KV_BYTES), dv = smem_u32(sV + s * KV_BYTES);
+            for (int r = lane; r < BN; r += 32) {
+                const int kj = j * BN + r;
+                const bool ok = kj < nk;
+                const int key = ok ? (a.indices ? a.indices[loff + kj] : kj) : 0;
+                const __nv_bfloat16 *srck = a.kr + (base + key) * D;
+                const __nv_bfloat16 *srcv = a.v + (base + key) * D;
+#pragma unroll
+                for (int ch = 0; ch < D / 8; ++ch) {
+                    cp_async16(dk + sw_off(r, ch, BN), srck + ch * 8, ok);
+                    cp_async16(dv + sw_off(r, ch, BN), srcv + ch * 8, ok);
+                }
+            }
+            cp_async_commit();
+            cp_async_wait_all();
+            fence_async_smem();
+            mbar_arrive(&bar_kv_full[s]);
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_qk = idesc_bf16(BN, false);
+            const uint32_t id_pv = idesc_bf16(D, true);
+            const uint32_t sQa = smem_u32(sQ);
+            bool ok = mbar_wait(&bar_q, 0, abort_flag, a.err, 0x20) &&
+                      mbar_wait(&bar_kv_full[0], 0, abort_flag, a.err, 0x21);
+            if (ok) {
+                tc_fence_after();
+                for (int t = 0; t < (two ? 2 : 1); ++t) {
+                    const uint32_t sKa = smem_u32(sK);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * (BM * 128) + (k & 3) * 32;
+                        mma_ss(tmem + t * 128, sw128_desc(sQa + t * QT_BYTES + ko, 16, 1024),
+                               sw128_desc(sKa + (k >> 2) * (BN * 128) + (k & 3) * 32, 16, 1024), id_qk, k > 0);
+                    }
+                    mma_commit(&bar_s_full[t]);
+                }
+            }
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int s = j & 1;
+                const uint32_t sVa = smem_u32(sV + s * KV_BYTES);
+                for (int t = 0; t < (two ? 2 : 1); ++t) {
+                    if (!mbar_wait(&bar_p_full[t], j & 1, abort_flag, a.err, 0x22)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < BN / 16; ++k)
+                        mma_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8,
+                               sw128_desc(sVa + k * 2048, BN * 128, 1024), id_pv, (j > 0 || k > 0));
+                    if (j + 1 < ntiles) {
+                        if (t == 0 && !mbar_wait(&bar_kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.err,
+                                                 0x23)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t sKa = smem_u32(sK + ((j + 1) & 1) * KV_BYTES);
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k) {
+                            const uint32_t ko = (k >> 2) * (BM * 128) + (k & 3) * 32;
+                            mma_ss(tmem + t * 128, sw128_desc(sQa + t * QT_BYTES + ko, 16, 1024),
+                                   sw128_desc(sKa + (k >> 2) * (BN * 128) + (k & 3) * 32, 16, 1024), id_qk,
+                                   k > 0);
+                        }
+                        mma_commit(&bar_s_full[t]);
+                    } else {
+                        mma_commit(&bar_o_final[t]);
+                    }
+                }
+                if (ok) mma_commit(&bar_kv_empty[s]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int t = warp >> 2;           // Q tile of this warpgroup
+        const int wq = warp & 3;           // TMEM lane quarter
+        const int row = wq * 32 + lane;    // row of the Q tile
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_off + t * 128;
+        const uint32_t tO = tmem + lane_off + 256 + t * 128;
+        const bool active = t == 0 || two;
+        float m_run = -INFINITY, l = 0.f;
+        bool ok = active;
+        for (int j = 0; ok && j < ntiles; ++j) {
+            if (!mbar_wait(&bar_s_full[t], j & 1, abort_flag, a.err, 0x30 + t)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sr[BN];
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + ch * 32, sr + ch * 32);
+            tmem_wait_ld();
+            const int valid = min(BN, nk - j * BN);
+            float s[BN];
+            float mt = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < BN; ++i) {
+                s[i] = i < valid ? __uint_as_float(sr[i]) * a.scale_log2 : -INFINITY;
+                mt = fmaxf(mt, s[i]);
+            }
+            if (j == 0) {
+                m_run = mt;
+            } else if (__any_sync(0xffffffffu, mt > m_run + 8.f)) {
+                const float mn = fmaxf(m_run, mt);
+                const float alpha = ex2(m_run - mn);
+                m_run = mn;
+                l *= alpha;
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + ch * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + ch * 32, o);
+                }
+            }
+            uint32_t p[BN / 2];
+#pragma unroll
+            for (int i = 0; i < BN / 2; ++i) {
+                const float p0 = ex2(s[2 * i] - m_run), p1 = ex2(s[2 * i + 1] - m_run);
+                l += p0 + p1;
+                p[i] = pack_bf16(p0, p1);
+            }
+            tmem_st32(tS, p);
+            tmem_st32(tS + 32, p + 32);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar_p_full[t]);
+        }
+        if (ok && mbar_wait(&bar_o_final[t], 0, abort_flag, a.err, 0x38 + t)) {
+            tc_fence_after();
+            const int qi = t * BM + row;
+            const bool store = qi < nq;
+            const int tok = store ? (a.perm ? a.perm[base + cstart + q0 + qi] : q0 + qi) : 0;
+            const float inv = 1.f / l;
+            __nv_bfloat16 *dst = a.o + (base + tok) * D;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(tO + ch * 32, o);
+                tmem_wait_ld();
+                if (store) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 u;
+                        u.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+                        u.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                        u.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+                        u.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(dst + ch * 32 + i) = u;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    }
+}
+
+// Work items: per (bh, cluster) ceil(|c| / 256) items of up to 256 queries
+// (dense: per bh, ceil(N / 256) contiguous items).
+__global__ void __launch_bounds__(1024) tc_items_kernel(const int32_t *sizes, int4 *items, int32_t *n_items, int BH,
+                                                        int Cq, int N)
+{
+    __shared__ int tmp[33];
+    int carry = 0;
+    for (int bh = 0; bh < BH; ++bh) {
+        for (int b0 = 0; b0 < Cq; b0 += blockDim.x) {
+            const int c = b0 + threadIdx.x;
+            const int sz = c < Cq ? (sizes ? sizes[(int64_t)bh * Cq + c] : N) : 0;
+            const int nt = (sz + 2 * BM - 1) / (2 * BM);
+            int tot;
+            const int ex = block_excl_scan(nt, tmp, tot);
+            for (int t = 0; t < nt; ++t) {
+                const int q0 = t * 2 * BM;
+                items[carry + ex + t] = make_int4(bh, c, q0, min(2 * BM, sz - q0));
+            }
+            carry += tot;
+        }
+    }
+    if (threadIdx.x == 0) *n_items = carry;
+}
+
+}  // namespace tc
+
+constexpr size_t tc_smem_bytes(int D) { return (size_t)(2 * tc::BM * D * 2 + 4 * tc::BN * D * 2) + 1024; }
+
+cudaError_t attn_tc_configure()
+{
+    cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tc_smem_bytes(128));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(tc::attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)tc_smem_bytes(64));
+}
+
+int attn_tc_max_items(int BH, int N, int Cq) { return BH * ((N + 2 * tc::BM - 1) / (2 * tc::BM) + Cq); }
+
+void launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv_bfloat16 *v, __nv_bfloat16 *o,
+                    int4 *items, int32_t *n_items, int max_items, const int32_t *sizes, const int32_t *perm,
+                    const int32_t *start, const long long *offsets, const int32_t *indices, const int32_t *n_c,
+                    int32_t *err, int BH, int N, int D, int Cq, cudaStream_t st)
+{
+    tc::tc_items_kernel<<<1, 1024, 0, st>>>(sizes, items, n_items, BH, sizes ? Cq : 1, N);
+    count_launches(1);
+    tc::Args a;
+    a.qr = qr;
+    a.kr = kr;
+    a.v = v;
+    a.o = o;
+    a.items = items;
+    a.n_items = n_items;
+    a.perm = perm;
+    a.start = start;
+    a.offsets = offsets;
+    a.indices = indices;
+    a.n_c = n_c;
+    a.err = err;
+    a.N = N;
+    a.Cq = Cq;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+    if (D == 128)
+        tc::attn_tc_kernel<128><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(a);
+    else
+        tc::attn_tc_kernel<64><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(a);
+    count_launches(1);
+}
+
+}  // namespace scope

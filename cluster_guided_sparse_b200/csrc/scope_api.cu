@@ -28,10 +28,11 @@ void launch_lut(const float *, const float *, const float *, const float *, floa
                 int, int, int, cudaStream_t);
 void launch_items(const int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, int, int, int, int, int, int,
                   cudaStream_t);
-void launch_tiles(const int32_t *, int2 *, int32_t *, int, int, int, cudaStream_t);
-void launch_attn_simt(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, __nv_bfloat16 *,
-                      const int2 *, const int32_t *, int, const int32_t *, const int32_t *, const long long *,
-                      const int32_t *, const int32_t *, int, int, int, int, cudaStream_t);
+cudaError_t attn_tc_configure();
+int attn_tc_max_items(int BH, int N, int Cq);
+void launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, __nv_bfloat16 *, int4 *,
+                    int32_t *, int, const int32_t *, const int32_t *, const int32_t *, const long long *,
+                    const int32_t *, const int32_t *, int32_t *, int, int, int, int, cudaStream_t);
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
                    const int32_t *item_n, int Pcap, int N, int Cq, int Ct, int Ch, int Cw, int BH, float top_p,
                    float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes, int32_t *r, int32_t *n,
@@ -68,12 +69,12 @@ namespace {
 
 struct Layout {
     int64_t B, H, N, D, BH;
-    int Cq, C[3], ds[3], off[3], Csum, P, Pcap, nblk, max_tiles, maxL, maxP;
+    int Cq, C[3], ds[3], off[3], Csum, P, Pcap, nblk, max_work, maxL, maxP;
     bool f32, bisect;
     int64_t cap;
     size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
-    size_t lut, item_hist, item_id, item_cnt, item_n, r, n, kh, offsets, indices, tiles, ntiles, vb;
+    size_t lut, item_hist, item_id, item_cnt, item_n, r, n, kh, offsets, indices, work, nwork, vb;
     size_t total;
 };
 
@@ -191,7 +192,7 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.P = L.C[0] * L.C[1] * L.C[2];
     L.Pcap = (int)(L.P < L.N ? L.P : L.N);
     L.nblk = (int)((L.N + kSortBlk - 1) / kSortBlk);
-    L.max_tiles = (int)((L.N + kTQ - 1) / kTQ) + L.Cq;
+    L.max_work = attn_tc_max_items((int)L.BH, (int)L.N, L.Cq);
     const int T = g ? g->T : 0, Hh = g ? g->Hh : 0, W = g ? g->W : 0;
     L.maxL = T > Hh ? T : Hh;
     L.maxL = L.maxL > W ? L.maxL : W;
@@ -231,8 +232,8 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.n = take(cur, BH * L.Cq * 4);
     L.kh = take(cur, BH * 4);
     L.offsets = take(cur, (BH * L.Cq + 1) * 8);
-    L.tiles = take(cur, BH * L.max_tiles * 8);
-    L.ntiles = take(cur, BH * 4);
+    L.work = take(cur, (size_t)L.max_work * 16);
+    L.nwork = take(cur, 16);
     L.vb = take(cur, L.f32 ? BH * N * D * 2 : 0);
     L.indices = take(cur, (size_t)L.cap * 4);
     L.total = cur;
@@ -248,7 +249,8 @@ scope_status check_device(cudaStream_t)
     if (major != 10) return fail(SCOPE_EDEVICE, "libscope.so is built for sm_100a; device has compute capability %d.x", major);
     static bool configured[64] = {false};
     if (dev < 64 && !configured[dev]) {
-        if (km_configure() != cudaSuccess) return fail(SCOPE_ECUDA, "kernel attribute setup failed");
+        if (km_configure() != cudaSuccess || attn_tc_configure() != cudaSuccess)
+            return fail(SCOPE_ECUDA, "kernel attribute setup failed");
         configured[dev] = true;
     }
     return SCOPE_OK;
@@ -392,8 +394,6 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
                   BH, p->top_p, 1.0f / sqrtf((float)D), p->k_min, at<int32_t>(ws, L.stats) + 4,
                   at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.r), at<int32_t>(ws, L.n), at<int32_t>(ws, L.kh),
                   at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, s);
-    launch_tiles(at<int32_t>(ws, L.q_sizes), at<int2>(ws, L.tiles), at<int32_t>(ws, L.ntiles), BH, L.Cq, L.max_tiles,
-                 s);
     if ((st = launch_status("selection")) != SCOPE_OK) return st;
 
     scope_plan_s *h = (scope_plan_s *)malloc(sizeof(scope_plan_s));
@@ -444,10 +444,11 @@ extern "C" scope_status scope_attn(const scope_tensor *q, const scope_tensor *k,
     if ((st = check_device(s)) != SCOPE_OK) return st;
     char *ws = plan->ws;
     const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
-    launch_attn_simt(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
-                     at<int2>(ws, L.tiles), at<int32_t>(ws, L.ntiles), L.max_tiles, at<int32_t>(ws, L.q_perm),
-                     at<int32_t>(ws, L.q_start), at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices),
-                     at<int32_t>(ws, L.n), (int)L.BH, (int)L.N, (int)L.D, L.Cq, s);
+    launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
+                   at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, at<int32_t>(ws, L.q_sizes),
+                   at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start), at<long long>(ws, L.offsets),
+                   at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n), at<int32_t>(ws, L.stats) + 4, (int)L.BH,
+                   (int)L.N, (int)L.D, L.Cq, s);
     return launch_status("scope_attn");
 }
 
@@ -471,6 +472,9 @@ static Layout dense_layout(const scope_tensor *q, const scope_grid *g, const sco
     L.tab = take(cur, (size_t)3 * L.maxL * L.maxP * 16);
     L.stats = take(cur, 64);
     L.vb = take(cur, L.f32 ? L.BH * L.N * L.D * 2 : 0);
+    L.max_work = attn_tc_max_items((int)L.BH, (int)L.N, 0);
+    L.work = take(cur, (size_t)L.max_work * 16);
+    L.nwork = take(cur, 16);
     L.total = cur;
     return L;
 }
@@ -517,8 +521,9 @@ extern "C" scope_status scope_dense_attn(const scope_tensor *q, const scope_tens
     char *ws = (char *)workspace;
     rope_both(L, ws, q, k, has_grid ? grid : nullptr, p, s);
     const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
-    launch_attn_simt(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr, nullptr,
-                     nullptr, 0, nullptr, nullptr, nullptr, nullptr, nullptr, (int)L.BH, (int)L.N, (int)L.D, 1, s);
+    launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
+                   at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, nullptr, nullptr, nullptr, nullptr,
+                   nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, (int)L.BH, (int)L.N, (int)L.D, 1, s);
     return launch_status("scope_dense_attn");
 }
 
