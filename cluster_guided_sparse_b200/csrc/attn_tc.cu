@@ -6,12 +6,16 @@
 // of 128 keys.  Both Q tiles share every gathered K/V tile, which halves the
 // K/V bytes per flop (the tiles come from L2: a head's K/V is 61 MB at 720p).
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3  softmax / epilogue of Q tile 0 (one thread per query row)
 //   warps 4-7  softmax / epilogue of Q tile 1
 //   warp 8     tcgen05.mma issuer (one lane), owns the TMEM allocation
-//   warp 9     producer: gathers Q rows and the listed K/V rows with 16-byte
-//              cp.async into 128B-swizzled shared-memory tiles (2 stages)
+//   warps 9-10 producer: Q rows and the listed K and V rows by coalesced
+//              16-byte cp.async (16 lanes per 256-byte row) into 128B-swizzled
+//              shared-memory tiles, 2 stages each; K and V have their own
+//              full/empty barriers so K(j+1) can land while V(j) is in use.
+//              (A tile::gather4 TMA producer measured ~7 B/clk per SM here,
+//              which made the loads the bottleneck; the LSU gather does not.)
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
 // S = Q K^T lands in TMEM (fp32); the softmax rows read it with tcgen05.ld,
 // write P as packed bf16 over the first 64 columns of their S, and the
@@ -19,17 +23,25 @@
 // Online softmax in base 2 with a lazy rescale: O and l are rescaled only
 // when a row's max grows by more than 2^8, so P never exceeds 256.
 //
+// The softmax loads its 128-wide S row with four back-to-back tcgen05.ld
+// (one wait) for the row max, reloads it in two halves for the exponentials,
+// and does the scale/subtract and the row sum with packed f32x2 instructions.
+// (Moving a third of the exponentials to a cubic on the FMA pipe was slower
+// here: the softmax is latency-bound, not MUFU-bound.)
+//
 // Every mbarrier wait is bounded (about two seconds of clock64); on timeout
 // the thread records SCOPE's timeout bit in the device error word, the CTA
 // abandons its work item, and all threads still meet at the final barrier
 // so the TMEM is released.
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace scope {
 
 namespace tc {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int BN = 128;       // keys per K/V tile
 constexpr int BM = 128;       // rows per Q tile
 constexpr long long kWaitCycles = 4000000000ll;
@@ -76,6 +88,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
             }
         }
     }
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Four rows (y0..y3) x 64 bf16 columns starting at column x, 512 bytes.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *tm, int x, int y0, int y1, int y2,
+                                            int y3, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
+        : "memory");
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
@@ -156,8 +185,39 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// d = a * b + c on a pair of fp32 values (one f32x2 instruction).
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0, float c1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.ftz.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void fadd2(float &d0, float &d1, float a0, float a1)
+{
+    asm("{\n\t.reg .b64 ra, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+        "add.rn.ftz.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1));
+}
+
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ float ex2(float x)
 {
@@ -195,7 +255,8 @@ struct Args {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Args a)
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Args a)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzle atoms.
@@ -206,7 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Args a)
     unsigned char *sK = sm + 2 * QT_BYTES;       // 2 stages
     unsigned char *sV = sK + 2 * KV_BYTES;       // 2 stages
 
-    __shared__ uint64_t bar_q, bar_kv_full[2], bar_kv_empty[2], bar_s_full[2], bar_p_full[2], bar_o_final[2];
+    __shared__ uint64_t bar_q, bar_k_full[2], bar_k_empty[2], bar_v_full[2], bar_v_empty[2], bar_s_full[2],
+        bar_p_full[2], bar_o_final[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
 
@@ -223,10 +285,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Args a)
     const int ntiles = (nk + BN - 1) / BN;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bar_q, 32);
+        mbar_init(&bar_q, 64);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar_kv_full[i], 32);
-            mbar_init(&bar_kv_empty[i], 1);
+            mbar_init(&bar_k_full[i], 64);
+            mbar_init(&bar_k_empty[i], 1);
+            mbar_init(&bar_v_full[i], 64);
+            mbar_init(&bar_v_empty[i], 1);
             mbar_init(&bar_s_full[i], 1);
             mbar_init(&bar_p_full[i], 128);
             mbar_init(&bar_o_final[i], 1);
@@ -244,70 +308,101 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Args a)
     const uint32_t tmem = tmem_base_sh;
     volatile int *abort_flag = &abort_sh;
 
-    if (warp == 9) {
+    if (warp >= 9) {
         // ------------------------------------------------------------ producer
-        // Q rows (zero-filled past the work item's queries).
-        for (int t = 0; t < 2; ++t) {
-            const uint32_t dst0 = smem_u32(sQ + t * QT_BYTES);
-            for (int r = lane; r < BM; r += 32) {
-                const int qi = t * BM + r;
-                const bool ok = qi < nq;
-                const int tok = ok ? (a.perm ? a.perm[base + cstart + q0 + qi] : q0 + qi) : 0;
-                const __nv_bfloat16 *src = a.qr + (base + tok) * D;
-#pragma unroll
-                for (int ch = 0; ch < D / 8; ++ch) cp_async16(dst0 + sw_off(r, ch, BM), src + ch * 8, ok);
-            }
+        // 64 threads; a warp instruction covers 32 / (D/8) whole rows, so
+        // every 16-byte chunk request is part of a fully used 128-byte line.
+        constexpr int CH = D / 8;           // 16-byte chunks per row
+        constexpr int RPI = 64 / CH;         // rows per producer-wide pass
+        const int pt = threadIdx.x - 9 * 32;
+        const int ch = pt % CH, r0 = pt / CH;
+        for (int qi0 = 0; qi0 < 2 * BM; qi0 += RPI) {
+            const int qi = qi0 + r0, t = qi / BM, r = qi % BM;
+            const bool ok = qi < nq;
+            const int tok = ok ? (a.perm ? a.perm[base + cstart + q0 + qi] : q0 + qi) : 0;
+            cp_async16(smem_u32(sQ + t * QT_BYTES) + sw_off(r, ch, BM), a.qr + (base + tok) * D + ch * 8, ok);
         }
         cp_async_commit();
         cp_async_wait_all();
         fence_async_smem();
         mbar_arrive(&bar_q);
-        for (int j = 0; j < ntiles; ++j) {
-            const int s = j & 1;
-            if (j >= 2 && !mbar_wait(&bar_kv_empty[s], ((j >> 1) - 1) & 1, abort_flag, a.err, 0x10)) break;
-            const uint32_t dk = smem_u32(sK + s * KV_BYTES), dv = smem_u32(sV + s * KV_BYTES);
-            for (int r = lane; r < BN; r += 32) {
-                const int kj = j * BN + r;
-                const bool ok = kj < nk;
-                const int key = ok ? (a.indices ? a.indices[loff + kj] : kj) : 0;
-                const __nv_bfloat16 *srck = a.kr + (base + key) * D;
-                const __nv_bfloat16 *srcv = a.v + (base + key) * D;
+        // Rows past the list repeat the last listed key (finite V, masked P).
+        // A tile's keys are read once, up front (independent loads), and
+        // serve both its K and its V rows.
+        constexpr int NR = BN / RPI;
+        int keys[NR];
+        auto load_keys = [&](int j) {
 #pragma unroll
-                for (int ch = 0; ch < D / 8; ++ch) {
-                    cp_async16(dk + sw_off(r, ch, BN), srck + ch * 8, ok);
-                    cp_async16(dv + sw_off(r, ch, BN), srcv + ch * 8, ok);
-                }
+            for (int i = 0; i < NR; ++i) {
+                const int kj = min(j * BN + i * RPI + r0, nk - 1);
+                keys[i] = a.indices ? a.indices[loff + kj] : kj;
             }
+        };
+        auto issue = [&](unsigned char *dst_base, const __nv_bfloat16 *src, int j) {
+            const uint32_t dst = smem_u32(dst_base + (j & 1) * KV_BYTES);
+#pragma unroll
+            for (int i = 0; i < NR; ++i)
+                cp_async16(dst + sw_off(i * RPI + r0, ch, BN), src + (base + keys[i]) * D + ch * 8, true);
             cp_async_commit();
-            cp_async_wait_all();
+        };
+        load_keys(0);
+        issue(sK, a.kr, 0);
+        issue(sV, a.v, 0);
+        for (int j = 0; j < ntiles; ++j) {
+            const bool more = j + 1 < ntiles;
+            // in flight: K(j), V(j)
+            cp_async_wait1();
             fence_async_smem();
-            mbar_arrive(&bar_kv_full[s]);
+            mbar_arrive(&bar_k_full[j & 1]);
+            if (more) {
+                load_keys(j + 1);
+                if (j + 1 >= 2 && !mbar_wait(&bar_k_empty[(j + 1) & 1], (((j + 1) >> 1) - 1) & 1, abort_flag, a.err,
+                                             0x10))
+                    break;
+                issue(sK, a.kr, j + 1);
+                cp_async_wait1();  // in flight: V(j), K(j+1)
+            } else {
+                cp_async_wait_all();
+            }
+            fence_async_smem();
+            mbar_arrive(&bar_v_full[j & 1]);
+            if (more) {
+                if (j + 1 >= 2 && !mbar_wait(&bar_v_empty[(j + 1) & 1], (((j + 1) >> 1) - 1) & 1, abort_flag, a.err,
+                                             0x11))
+                    break;
+                issue(sV, a.v, j + 1);
+            }
         }
+        cp_async_wait_all();
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16(BN, false);
             const uint32_t id_pv = idesc_bf16(D, true);
             const uint32_t sQa = smem_u32(sQ);
+            const int nt = two ? 2 : 1;
+            auto issue_qk = [&](int t, int j) {
+                const uint32_t sKa = smem_u32(sK + (j & 1) * KV_BYTES);
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t ko = (k >> 2) * (BM * 128) + (k & 3) * 32;
+                    mma_ss(tmem + t * 128, sw128_desc(sQa + t * QT_BYTES + ko, 16, 1024),
+                           sw128_desc(sKa + (k >> 2) * (BN * 128) + (k & 3) * 32, 16, 1024), id_qk, k > 0);
+                }
+                mma_commit(&bar_s_full[t]);
+                if (t == nt - 1) mma_commit(&bar_k_empty[j & 1]);
+            };
             bool ok = mbar_wait(&bar_q, 0, abort_flag, a.err, 0x20) &&
-                      mbar_wait(&bar_kv_full[0], 0, abort_flag, a.err, 0x21);
+                      mbar_wait(&bar_k_full[0], 0, abort_flag, a.err, 0x21);
             if (ok) {
                 tc_fence_after();
-                for (int t = 0; t < (two ? 2 : 1); ++t) {
-                    const uint32_t sKa = smem_u32(sK);
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t ko = (k >> 2) * (BM * 128) + (k & 3) * 32;
-                        mma_ss(tmem + t * 128, sw128_desc(sQa + t * QT_BYTES + ko, 16, 1024),
-                               sw128_desc(sKa + (k >> 2) * (BN * 128) + (k & 3) * 32, 16, 1024), id_qk, k > 0);
-                    }
-                    mma_commit(&bar_s_full[t]);
-                }
+                for (int t = 0; t < nt; ++t) issue_qk(t, 0);
             }
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int s = j & 1;
+                if (!mbar_wait(&bar_v_full[s], (j >> 1) & 1, abort_flag, a.err, 0x24)) break;
                 const uint32_t sVa = smem_u32(sV + s * KV_BYTES);
-                for (int t = 0; t < (two ? 2 : 1); ++t) {
+                for (int t = 0; t < nt; ++t) {
                     if (!mbar_wait(&bar_p_full[t], j & 1, abort_flag, a.err, 0x22)) {
                         ok = false;
                         break;
@@ -317,26 +412,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Args a)
                     for (int k = 0; k < BN / 16; ++k)
                         mma_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8,
                                sw128_desc(sVa + k * 2048, BN * 128, 1024), id_pv, (j > 0 || k > 0));
+                    if (t == nt - 1) mma_commit(&bar_v_empty[s]);
                     if (j + 1 < ntiles) {
-                        if (t == 0 && !mbar_wait(&bar_kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.err,
+                        if (t == 0 && !mbar_wait(&bar_k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.err,
                                                  0x23)) {
                             ok = false;
                             break;
                         }
-                        const uint32_t sKa = smem_u32(sK + ((j + 1) & 1) * KV_BYTES);
-#pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {
-                            const uint32_t ko = (k >> 2) * (BM * 128) + (k & 3) * 32;
-                            mma_ss(tmem + t * 128, sw128_desc(sQa + t * QT_BYTES + ko, 16, 1024),
-                                   sw128_desc(sKa + (k >> 2) * (BN * 128) + (k & 3) * 32, 16, 1024), id_qk,
-                                   k > 0);
-                        }
-                        mma_commit(&bar_s_full[t]);
+                        issue_qk(t, j + 1);
                     } else {
                         mma_commit(&bar_o_final[t]);
                     }
                 }
-                if (ok) mma_commit(&bar_kv_empty[s]);
             }
         }
         __syncwarp();
@@ -357,44 +444,84 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(Args a)
                 break;
             }
             tc_fence_after();
-            uint32_t sr[BN];
-#pragma unroll
-            for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + ch * 32, sr + ch * 32);
-            tmem_wait_ld();
             const int valid = min(BN, nk - j * BN);
-            float s[BN];
-            float mt = -INFINITY;
+            uint32_t r[BN];
 #pragma unroll
-            for (int i = 0; i < BN; ++i) {
-                s[i] = i < valid ? __uint_as_float(sr[i]) * a.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, s[i]);
+            for (int c4 = 0; c4 < BN / 32; ++c4) tmem_ld32(tS + c4 * 32, r + c4 * 32);
+            tmem_wait_ld();
+            if (valid < BN) {
+#pragma unroll
+                for (int i = 0; i < BN; ++i)
+                    if (i >= valid) r[i] = __float_as_uint(-INFINITY);
             }
+            float m8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(r[i]);
+#pragma unroll
+            for (int i = 8; i < BN; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(r[i]));
+            const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            const float mt = mraw * a.scale_log2;
+            // Lazy rescale: move the reference max only when it grew by > 8
+            // (log2 units); O and l are scaled after P is written, so the S
+            // row and the O chunk never need registers at the same time.
+            bool rescale = false;
+            float alpha = 1.f;
             if (j == 0) {
                 m_run = mt;
             } else if (__any_sync(0xffffffffu, mt > m_run + 8.f)) {
                 const float mn = fmaxf(m_run, mt);
-                const float alpha = ex2(m_run - mn);
+                alpha = ex2(m_run - mn);
                 m_run = mn;
                 l *= alpha;
+                rescale = true;
+            }
+            // p = 2^(s*scale - m) on pairs, reloading S in two 64-column halves;
+            // row sum in two lanes; bf16 pairs written over S.
+            const float nm = -m_run, sc = a.scale_log2;
+            float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t q[64];
+                tmem_ld32(tS + h2 * 64, q);
+                tmem_ld32(tS + h2 * 64 + 32, q + 32);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c4 = 0; c4 < 2; ++c4) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int col = h2 * 64 + c4 * 32 + 2 * i;
+                        float x0, x1, p0, p1;
+                        ffma2(x0, x1, __uint_as_float(q[c4 * 32 + 2 * i]), __uint_as_float(q[c4 * 32 + 2 * i + 1]), sc,
+                              sc, nm, nm);
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
+                        if (valid < BN) {
+                            p0 = col < valid ? p0 : 0.f;
+                            p1 = col + 1 < valid ? p1 : 0.f;
+                        }
+                        if (i & 1) fadd2(lc, ld, p0, p1);
+                        else fadd2(la, lb, p0, p1);
+                        pk[i] = pack_bf16(p0, p1);
+                    }
+                    tmem_st16(tS + h2 * 32 + c4 * 16, pk);
+                }
+            }
+            la += lc;
+            lb += ld;
+            l += la + lb;
+            if (rescale) {
+#pragma unroll
+                for (int c4 = 0; c4 < D / 32; ++c4) {
                     uint32_t o[32];
-                    tmem_ld32(tO + ch * 32, o);
+                    tmem_ld32(tO + c4 * 32, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tO + ch * 32, o);
+                    tmem_st32(tO + c4 * 32, o);
                 }
             }
-            uint32_t p[BN / 2];
-#pragma unroll
-            for (int i = 0; i < BN / 2; ++i) {
-                const float p0 = ex2(s[2 * i] - m_run), p1 = ex2(s[2 * i + 1] - m_run);
-                l += p0 + p1;
-                p[i] = pack_bf16(p0, p1);
-            }
-            tmem_st32(tS, p);
-            tmem_st32(tS + 32, p + 32);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bar_p_full[t]);
@@ -472,11 +599,39 @@ cudaError_t attn_tc_configure()
 
 int attn_tc_max_items(int BH, int N, int Cq) { return BH * ((N + 2 * tc::BM - 1) / (2 * tc::BM) + Cq); }
 
-void launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv_bfloat16 *v, __nv_bfloat16 *o,
+// Tensor map over the rows of a [rows][D] bf16 tensor: box of 64 columns x 1
+// row (the tile::gather4 form), 128-byte swizzle.
+static bool rows_tensor_map(CUtensorMap *m, const void *base, uint64_t rows, int D)
+{
+    using Encode = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static Encode encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return false;
+        encode = (Encode)fn;
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv_bfloat16 *v, __nv_bfloat16 *o,
                     int4 *items, int32_t *n_items, int max_items, const int32_t *sizes, const int32_t *perm,
                     const int32_t *start, const long long *offsets, const int32_t *indices, const int32_t *n_c,
                     int32_t *err, int BH, int N, int D, int Cq, cudaStream_t st)
 {
+    CUtensorMap tmK, tmV;
+    if (!rows_tensor_map(&tmK, kr, (uint64_t)BH * N, D) || !rows_tensor_map(&tmV, v, (uint64_t)BH * N, D))
+        return false;
     tc::tc_items_kernel<<<1, 1024, 0, st>>>(sizes, items, n_items, BH, sizes ? Cq : 1, N);
     count_launches(1);
     tc::Args a;
@@ -496,10 +651,11 @@ void launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv
     a.Cq = Cq;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     if (D == 128)
-        tc::attn_tc_kernel<128><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(a);
+        tc::attn_tc_kernel<128><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(tmK, tmV, a);
     else
-        tc::attn_tc_kernel<64><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(a);
+        tc::attn_tc_kernel<64><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(tmK, tmV, a);
     count_launches(1);
+    return true;
 }
 
 }  // namespace scope

@@ -102,6 +102,199 @@ __global__ void __launch_bounds__(128) km_assign_direct_kernel(KmBatch b, int N,
     if (n < N) P.labels[(int64_t)bh * N + n] = arg;
 }
 
+// -------------------------------------------------------------- assign (tiled, certified)
+// Query assignment for C >= 128: each CTA scores 128 rows against all
+// centroids in 128-wide chunks with 8x8 register tiles per thread, using the
+// expanded form e_j = ||c_j||^2 - 2 x.c_j (one FMA per row-centroid-dim).
+// The fp32 error of every e_j is at most
+//   B = (dim + 2) * 2^-24 * (2 |x| R + R^2),   R = max_j |c_j|
+// (dot-product and norm rounding bounds), so if the runner-up beats the best
+// by more than 2B the argmin is certain; rows inside the margin (and exact
+// ties) are listed and re-decided by km_fixup_kernel in fp64 on the direct
+// form.  The labels are thus those of exact arithmetic on the stored fp32
+// centroids and bf16 rows.
+constexpr int kTP = 128, kTC = 128, kKS = 32;
+
+__device__ __forceinline__ void better(float &b1, int &a1, float &b2, float e, int j)
+{
+    if (e < b1 || (e == b1 && j < a1)) {
+        b2 = b1;
+        b1 = e;
+        a1 = j;
+    } else if (e < b2) {
+        b2 = e;
+    }
+}
+
+__global__ void __launch_bounds__(256, 2) km_assign_tiled_kernel(KmProblem P, int N, int D, const float *xnorm2,
+                                                                 int32_t *fix_list, int32_t *fix_count)
+{
+    extern __shared__ __align__(16) float smt[];
+    float *xs = smt;               // [kKS][kTP]
+    float *cs = smt + kKS * kTP;   // [kKS][kTC]
+    __shared__ float red[8];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int bh = blockIdx.y, p0 = blockIdx.x * kTP;
+    const int C = P.C, dn = P.dim_n;
+    const __nv_bfloat16 *X = P.X + (int64_t)bh * N * D + P.dim_off;
+    const float *cent = P.cent + (int64_t)bh * C * dn;
+    const float *cn = P.cn + (int64_t)bh * C;
+
+    // R^2 = max_j |c_j|^2
+    float r2 = 0.f;
+    for (int j = tid; j < C; j += 256) r2 = fmaxf(r2, cn[j]);
+    r2 = warp_max(r2);
+    if ((tid & 31) == 0) red[tid >> 5] = r2;
+    __syncthreads();
+    r2 = red[0];
+    for (int i = 1; i < 8; ++i) r2 = fmaxf(r2, red[i]);
+
+    float b1[8], b2[8];
+    int a1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        b1[i] = INFINITY;
+        b2[i] = INFINITY;
+        a1[i] = 0;
+    }
+    for (int c0 = 0; c0 < C; c0 += kTC) {
+        float acc[8][8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+        for (int k0 = 0; k0 < dn; k0 += kKS) {
+            __syncthreads();
+            // rows: 128 x 32 bf16 -> xs[k][p]; each thread one 8-wide piece, twice
+            for (int idx = tid; idx < kTP * (kKS / 8); idx += 256) {
+                const int p = idx >> 2, k8 = (idx & 3) * 8, n = p0 + p;
+                float v[8];
+                if (n < N) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(X + (int64_t)n * D + k0 + k8);
+                    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 f = __bfloat1622float2(h[q]);
+                        v[2 * q] = f.x;
+                        v[2 * q + 1] = f.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) v[q] = 0.f;
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) xs[(k8 + q) * kTP + p] = v[q];
+            }
+            // centroids: 128 x 32 fp32 -> cs[k][c]
+            for (int idx = tid; idx < kTC * (kKS / 4); idx += 256) {
+                const int c = idx >> 3, k4 = (idx & 7) * 4;
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (c0 + c < C) v = *reinterpret_cast<const float4 *>(cent + (int64_t)(c0 + c) * dn + k0 + k4);
+                cs[(k4 + 0) * kTC + c] = v.x;
+                cs[(k4 + 1) * kTC + c] = v.y;
+                cs[(k4 + 2) * kTC + c] = v.z;
+                cs[(k4 + 3) * kTC + c] = v.w;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int k = 0; k < kKS; ++k) {
+                const float4 x0 = *reinterpret_cast<const float4 *>(xs + k * kTP + ty * 8);
+                const float4 x1 = *reinterpret_cast<const float4 *>(xs + k * kTP + ty * 8 + 4);
+                const float4 w0 = *reinterpret_cast<const float4 *>(cs + k * kTC + tx * 8);
+                const float4 w1 = *reinterpret_cast<const float4 *>(cs + k * kTC + tx * 8 + 4);
+                const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                const float cv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xv[i], cv[j], acc[i][j]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int c = c0 + tx * 8 + j;
+            if (c < C) {
+                const float cnj = cn[c];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) better(b1[i], a1[i], b2[i], fmaf(-2.f, acc[i][j], cnj), c);
+            }
+        }
+    }
+    // merge over the 16 lanes that share these rows
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float ob1 = __shfl_xor_sync(0xffffffffu, b1[i], o);
+            const float ob2 = __shfl_xor_sync(0xffffffffu, b2[i], o);
+            const int oa1 = __shfl_xor_sync(0xffffffffu, a1[i], o);
+            better(b1[i], a1[i], b2[i], ob1, oa1);
+            b2[i] = fminf(b2[i], ob2);
+        }
+    }
+    if (tx < 8) {
+        const int i = tx;
+        const int n = p0 + ty * 8 + i;
+        float bb1 = b1[0], bb2 = b2[0];
+        int aa = a1[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+            if (q == i) {
+                bb1 = b1[q];
+                bb2 = b2[q];
+                aa = a1[q];
+            }
+        if (n < N) {
+            const float xn = sqrtf(xnorm2[(int64_t)bh * N + n]);
+            const float R = sqrtf(r2);
+            const float B = (float)(dn + 2) * 5.9604645e-8f * (2.f * xn * R + r2) * 1.01f + 1e-30f;
+            P.labels[(int64_t)bh * N + n] = aa;
+            if (!(bb2 - bb1 > 2.f * B)) {
+                const int slot = atomicAdd(fix_count, 1);
+                fix_list[slot] = bh * N + n;
+            }
+        }
+    }
+}
+
+// Exact re-decision of the listed rows: fp64 direct-form distance to every
+// centroid, lowest index on ties.  One warp per row.
+__global__ void __launch_bounds__(256) km_fixup_kernel(KmProblem P, int N, int D, const int32_t *fix_list,
+                                                       const int32_t *fix_count)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    const int count = *fix_count;
+    const int C = P.C, dn = P.dim_n;
+    for (int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < count; w += warps) {
+        const int gid = fix_list[w];
+        const int bh = gid / N, n = gid % N;
+        const __nv_bfloat16 *x = P.X + ((int64_t)bh * N + n) * D + P.dim_off;
+        double xv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xv[q] = lane + 32 * q < dn ? (double)__bfloat162float(x[lane + 32 * q]) : 0.0;
+        const float *cent = P.cent + (int64_t)bh * C * dn;
+        double best = INFINITY;
+        int arg = 0;
+        for (int j = 0; j < C; ++j) {
+            double d = 0.0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (lane + 32 * q < dn) {
+                    const double t = xv[q] - (double)cent[(int64_t)j * dn + lane + 32 * q];
+                    d = fma(t, t, d);
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+            if (d < best) {
+                best = d;
+                arg = j;
+            }
+        }
+        if (lane == 0) P.labels[(int64_t)bh * N + n] = arg;
+    }
+}
+
 // -------------------------------------------------------------- stable counting sort
 // One warp per block of kSortBlk consecutive rows.
 __global__ void km_hist_kernel(KmBatch b, int N, int nblk)
@@ -229,8 +422,11 @@ static int max_dim(const KmBatch &b)
 
 cudaError_t km_configure()
 {
-    return cudaFuncSetAttribute(km_assign_direct_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (128 + 32) * 128 * 4);
+    cudaError_t e = cudaFuncSetAttribute(km_assign_direct_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (128 + 32) * 128 * 4);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(km_assign_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                2 * kKS * kTP * (int)sizeof(float));
 }
 
 void launch_km_init(const KmBatch &b, int BH, int N, int D, uint32_t seed, cudaStream_t st)
@@ -244,6 +440,17 @@ void launch_km_assign_direct(const KmBatch &b, int BH, int N, int D, cudaStream_
     const int dn = max_dim(b);
     const size_t smem = (size_t)(128 + 32) * dn * sizeof(float);
     km_assign_direct_kernel<32><<<dim3((N + 127) / 128, BH, b.count), 128, smem, st>>>(b, N, D);
+    count_launches(1);
+}
+
+void launch_km_assign_tiled(const KmProblem &P, int BH, int N, int D, const float *xnorm2, int32_t *fix_list,
+                            int32_t *fix_count, cudaStream_t st)
+{
+    cudaMemsetAsync(fix_count, 0, sizeof(int32_t), st);
+    km_assign_tiled_kernel<<<dim3((N + kTP - 1) / kTP, BH), 256, 2 * kKS * kTP * sizeof(float), st>>>(
+        P, N, D, xnorm2, fix_list, fix_count);
+    count_launches(1);
+    km_fixup_kernel<<<148 * 4, 256, 0, st>>>(P, N, D, fix_list, fix_count);
     count_launches(1);
 }
 

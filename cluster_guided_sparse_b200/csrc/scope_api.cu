@@ -22,6 +22,9 @@ cudaError_t km_configure();
 void launch_km_init(const KmBatch &, int, int, int, uint32_t, cudaStream_t);
 void launch_km_assign_direct(const KmBatch &, int, int, int, cudaStream_t);
 void launch_km_sort(const KmBatch &, int, int, cudaStream_t);
+void launch_bisect(const __nv_bfloat16 *, int, int, int, int, int, int32_t *, int32_t *, double *, int32_t *, float *,
+                   float *, int32_t *, int32_t *, int32_t *, cudaStream_t);
+void launch_km_assign_tiled(const KmProblem &, int, int, int, const float *, int32_t *, int32_t *, cudaStream_t);
 void launch_km_reduce(const KmBatch &, int, int, int, cudaStream_t);
 struct SelArgs;
 void launch_lut(const float *, const float *, const float *, const float *, float *, int, int, int, int, int, int,
@@ -30,7 +33,7 @@ void launch_items(const int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, i
                   cudaStream_t);
 cudaError_t attn_tc_configure();
 int attn_tc_max_items(int BH, int N, int Cq);
-void launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, __nv_bfloat16 *, int4 *,
+bool launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, __nv_bfloat16 *, int4 *,
                     int32_t *, int, const int32_t *, const int32_t *, const int32_t *, const long long *,
                     const int32_t *, const int32_t *, int32_t *, int, int, int, int, cudaStream_t);
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
@@ -74,7 +77,8 @@ struct Layout {
     int64_t cap;
     size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
-    size_t lut, item_hist, item_id, item_cnt, item_n, r, n, kh, offsets, indices, work, nwork, vb;
+    size_t lut, item_hist, item_id, item_cnt, item_n, r, n, kh, offsets, indices, work, nwork, vb, fix;
+    size_t bis_order, bis_delta;
     size_t total;
 };
 
@@ -106,6 +110,10 @@ bool tensor_ok(const scope_tensor *t, const char *name, scope_status *st)
     }
     if (t->D != 64 && t->D != 128) {
         *st = fail(SCOPE_ESHAPE, "%s: head dim must be 64 or 128 (got %lld)", name, (long long)t->D);
+        return false;
+    }
+    if (t->B * t->H * t->N >= (int64_t)1 << 31) {
+        *st = fail(SCOPE_ESHAPE, "%s: B*H*N must be < 2^31", name);
         return false;
     }
     if (t->N > (1 << 24)) {
@@ -214,6 +222,9 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.q_perm = take(cur, BH * N * 4);
     L.q_start = take(cur, BH * (L.Cq + 1) * 4);
     L.q_bhist = take(cur, BH * L.Cq * L.nblk * 4);
+    L.fix = take(cur, BH * N * 4 + 16);
+    L.bis_order = take(cur, L.bisect ? 2 * BH * N * 4 : 0);
+    L.bis_delta = take(cur, L.bisect ? BH * N * 8 : 0);
     L.k_codes = take(cur, 3 * BH * N * 4);
     for (int s = 0; s < 3; ++s) {
         L.k_cent[s] = take(cur, BH * L.C[s] * (ds[s] > 0 ? ds[s] : 1) * 4);
@@ -359,7 +370,6 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     if (((uintptr_t)workspace) & 255) return fail(SCOPE_EALIGN, "workspace must be 256-byte aligned");
     if (ws_bytes < L.total)
         return fail(SCOPE_EWORKSPACE, "workspace too small: %zu < %zu bytes", ws_bytes, L.total);
-    if (L.bisect) return fail(SCOPE_EINVAL, "fixed_cluster_size: bisection path not built in this library version");
     cudaStream_t s = (cudaStream_t)stream;
     if ((st = check_device(s)) != SCOPE_OK) return st;
     char *ws = (char *)workspace;
@@ -367,21 +377,53 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
 
     rope_both(L, ws, q, k, grid, p, s);
 
+    if (L.bisect) {
+        // ClusterAttention variant: balanced bisection of queries and of keys
+        // into N / fixed_cluster_size clusters (one subspace = the full head dim).
+        const int leaf = p->fixed_cluster_size;
+        int32_t *ord = at<int32_t>(ws, L.bis_order);
+        launch_bisect(at<__nv_bfloat16>(ws, L.qr), BH, N, D, leaf, p->iters, ord, ord + (int64_t)BH * N,
+                      at<double>(ws, L.bis_delta), at<int32_t>(ws, L.q_lab), at<float>(ws, L.q_cent),
+                      at<float>(ws, L.q_cn), at<int32_t>(ws, L.q_start), at<int32_t>(ws, L.q_sizes),
+                      at<int32_t>(ws, L.q_perm), s);
+        launch_bisect(at<__nv_bfloat16>(ws, L.kr), BH, N, D, leaf, p->iters, ord, ord + (int64_t)BH * N,
+                      at<double>(ws, L.bis_delta), at<int32_t>(ws, L.k_codes), at<float>(ws, L.k_cent[0]),
+                      at<float>(ws, L.k_cn[0]), at<int32_t>(ws, L.k_start[0]), at<int32_t>(ws, L.k_sizes[0]),
+                      at<int32_t>(ws, L.k_perm[0]), s);
+        cudaMemsetAsync(at<int32_t>(ws, L.k_codes) + (int64_t)BH * N, 0, (size_t)2 * BH * N * 4, s);
+    } else {
+    // Key subspaces always, and the queries when they have few clusters, run
+    // as one batch on the direct-form kernel; queries with >= 128 clusters use
+    // the register-tiled certified kernel (plus its fp64 fix-up pass).
+    const bool tiled_q = L.Cq >= 128;
     KmBatch all{};
     for (int i = 0; i < 3; ++i) all.p[i] = key_problem(L, ws, i);
     all.p[3] = query_problem(L, ws);
     all.count = 4;
+    KmBatch keys = all;
+    keys.count = 3;
     KmBatch qonly{};
     qonly.p[0] = all.p[3];
     qonly.count = 1;
+    int32_t *fix_count = at<int32_t>(ws, L.fix);
+    int32_t *fix_list = fix_count + 4;
+    auto assign = [&]() {
+        if (tiled_q) {
+            launch_km_assign_direct(keys, BH, N, D, s);
+            launch_km_assign_tiled(all.p[3], BH, N, D, at<float>(ws, L.qnorm), fix_list, fix_count, s);
+        } else {
+            launch_km_assign_direct(all, BH, N, D, s);
+        }
+    };
     launch_km_init(all, BH, N, D, p->init_seed, s);
     for (int it = 0; it < p->iters; ++it) {
-        launch_km_assign_direct(all, BH, N, D, s);
+        assign();
         launch_km_sort(all, BH, N, s);
         launch_km_reduce(all, BH, N, D, s);
     }
-    launch_km_assign_direct(all, BH, N, D, s);
+    assign();
     launch_km_sort(qonly, BH, N, s);
+    }
     if ((st = launch_status("k-means")) != SCOPE_OK) return st;
 
     launch_lut(at<float>(ws, L.q_cent), at<float>(ws, L.k_cent[0]), at<float>(ws, L.k_cent[1]),
@@ -444,11 +486,12 @@ extern "C" scope_status scope_attn(const scope_tensor *q, const scope_tensor *k,
     if ((st = check_device(s)) != SCOPE_OK) return st;
     char *ws = plan->ws;
     const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
-    launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
+    if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
                    at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, at<int32_t>(ws, L.q_sizes),
                    at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start), at<long long>(ws, L.offsets),
                    at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n), at<int32_t>(ws, L.stats) + 4, (int)L.BH,
-                   (int)L.N, (int)L.D, L.Cq, s);
+                   (int)L.N, (int)L.D, L.Cq, s))
+        return fail(SCOPE_ECUDA, "scope_attn: tensor map encoding failed");
     return launch_status("scope_attn");
 }
 
@@ -521,9 +564,10 @@ extern "C" scope_status scope_dense_attn(const scope_tensor *q, const scope_tens
     char *ws = (char *)workspace;
     rope_both(L, ws, q, k, has_grid ? grid : nullptr, p, s);
     const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
-    launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
-                   at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, nullptr, nullptr, nullptr, nullptr,
-                   nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, (int)L.BH, (int)L.N, (int)L.D, 1, s);
+    if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
+                        at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, nullptr, nullptr, nullptr,
+                        nullptr, nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, (int)L.BH, (int)L.N, (int)L.D, 1, s))
+        return fail(SCOPE_ECUDA, "scope_dense_attn: tensor map encoding failed");
     return launch_status("scope_dense_attn");
 }
 

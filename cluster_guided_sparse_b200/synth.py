@@ -57,6 +57,10 @@ class Workload:
     k_min: int
     online_topk: int
     fixed_cluster_size: int
+    # (bt, bh, bw): tokens of one grid block share one component label, blocks
+    # draw their labels independently (objects occupying regions); None = every
+    # token draws its own label.
+    label_block: Optional[tuple] = None
 
     @property
     def torch_dtype(self):
@@ -149,6 +153,14 @@ def make_head(w: Workload, b: int, h: int, seed: int = 0, field=None):
     if w.zipf_alpha > 0:
         pm = (np.arange(M) + 1.0) ** (-w.zipf_alpha)
         lab = g_lab.choice(M, size=N, p=pm / pm.sum())
+    elif w.label_block is not None:
+        T, Hh, W = w.grid
+        lbt, lbh, lbw = w.label_block
+        nb = (-(-T // lbt), -(-Hh // lbh), -(-W // lbw))
+        n = np.arange(N)
+        t, y, x = n // (Hh * W), (n // W) % Hh, n % W
+        block = ((t // lbt) * nb[1] + y // lbh) * nb[2] + x // lbw
+        lab = g_lab.integers(0, M, size=nb[0] * nb[1] * nb[2])[block]
     else:
         lab = g_lab.integers(0, M, size=N)
     s = head_sigma(w, h) / np.sqrt(D)

@@ -245,3 +245,53 @@ def test_degenerate_identical_tokens_leave_clusters_empty():
     sel = get(0)
     np.testing.assert_allclose(P.np64(o[0, 0]), np.broadcast_to(v[0, 0].double().numpy()[sel].mean(0), (128, 64)),
                                atol=2e-2)
+
+
+def bisect_parity(w, heads, cl_sample=None, q_sample=None, seed=0):
+    rng = np.random.default_rng(seed)
+    q, k, v = synth.make_inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    pl = plan_of(w, qd, kd)
+    o = scope.attn(qd, kd, vd, pl)
+    torch.cuda.synchronize()
+    pl.sync_status()
+    N, D, leaf = w.N, w.D, w.fixed_cluster_size
+    C = N // leaf
+    wq = w.with_(c_q=C, c_sub=(C, 1, 1))
+    tc = P.TieCounter()
+    for h in heads:
+        qr, kr = P.np64(pl.view("qr")[0, h]), P.np64(pl.view("kr")[0, h])
+        np.testing.assert_array_equal(qr, q[0, h].double().numpy())  # no grid: identity
+        np.testing.assert_array_equal(kr, k[0, h].double().numpy())
+        qlab = pl.view("q_labels")[0, h].cpu().numpy()
+        codes = [pl.view("k_codes")[s, 0, h].cpu().numpy() for s in range(3)]
+        qcent, kcent = P.np64(pl.view("q_centroids")[0, h]), P.np64(pl.view("k_cent_t")[0, h])
+        for X, lab_gpu, cent_gpu in ((qr, qlab, qcent), (kr, codes[0], kcent)):
+            lab, cent, perm = oracle.bisect(X, leaf, w.iters)
+            assert (lab == lab_gpu).all(), f"bisection labels differ on {(lab != lab_gpu).sum()} rows"
+            np.testing.assert_allclose(cent_gpu, cent, rtol=0, atol=1e-6 * max(1.0, np.abs(cent).max()))
+        assert (codes[1] == 0).all() and (codes[2] == 0).all()
+        sizes = pl.view("q_sizes")[0, h].cpu().numpy()
+        assert (sizes == leaf).all()
+        assert (pl.view("q_perm")[0, h].cpu().numpy() == np.argsort(qlab, kind="stable")).all()
+        lut = pl.view("lut")[0, h].cpu().numpy()
+        P.check_lut(qcent, [kcent, np.zeros((1, 0)), np.zeros((1, 0))], (D, 0, 0), lut.astype(np.float64))
+        clusters = np.arange(C) if cl_sample is None else rng.choice(C, cl_sample, replace=False)
+        get = lists_fn(pl, w, h)
+        P.check_selection(lut, codes, sizes, pl.view("r")[0, h].cpu().numpy(), pl.view("kh")[0, h].item(),
+                          pl.view("n")[0, h].cpu().numpy(), get, wq, N, D, clusters, tc)
+        rows = np.arange(N) if q_sample is None else np.sort(rng.choice(N, q_sample, replace=False))
+        P.check_attention(qr, kr, v[0, h].double().numpy(), qlab, get, P.np64(o[0, h]), rows)
+    tc.assert_ok("bisection Top-p counts")
+
+
+def test_unstructured_bisection_parity():
+    w = synth.WORKLOADS["unstructured"]
+    bisect_parity(w, [0, w.H - 1], cl_sample=8, q_sample=48)
+
+
+@pytest.mark.parametrize("N,D,H", [(128, 64, 1), (512, 128, 2), (4096, 64, 1)])
+def test_bisection_small_shapes(N, D, H):
+    w = synth.WORKLOADS["unstructured"].with_(N=N, D=D, H=H, d_split=(D, 0, 0), components=16, k_min=32,
+                                               config_id=150 + N, c_q=N // 64, c_sub=(N // 64, 1, 1))
+    bisect_parity(w, range(H))
