@@ -26,6 +26,7 @@ void launch_bisect(const __nv_bfloat16 *, int, int, int, int, int, int32_t *, in
                    float *, int32_t *, int32_t *, int32_t *, cudaStream_t);
 void launch_km_assign_tiled(const KmProblem &, int, int, int, const float *, int32_t *, int32_t *, cudaStream_t);
 void launch_km_reduce(const KmBatch &, int, int, int, cudaStream_t);
+
 struct SelArgs;
 void launch_lut(const float *, const float *, const float *, const float *, float *, int, int, int, int, int, int,
                 int, int, int, cudaStream_t);
