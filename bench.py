@@ -46,6 +46,23 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def attn_traffic(heads: int):
+    """DRAM bytes of one sparse-attention launch, from the committed ncu capture
+    (profiles/attn_tc_traffic.json) scaled from its heads to `heads`; None if the
+    kernel source changed since the capture."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_tc_traffic.json")) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, "cluster_guided_sparse_b200", "csrc", "attn_tc.cu"), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except Exception:
+        return None
+    if sha != rec.get("kernel_source_sha256"):
+        return None
+    return rec["sparse_dram_bytes_per_launch_captured"] * heads / rec["captured_heads"]
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
 
@@ -280,6 +297,20 @@ def run_scope(args, world, rank, local):
     hbm, bf16, bf16_sus, src = peaks()
     achieved = attn_flops / (attn_ms * 1e-3) / 1e12
 
+    # this build's dense attention (RoPE + all keys) at the same shape, for context
+    od = torch.empty_like(o)
+    dense = []
+    for i in range(1 + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        scope.dense_attn(qd, kd, vd, params, grid, out=od)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:
+            dense.append(a.elapsed_time(b))
+    dense_ms = statistics.mean(dense)
+    del od
+
     # end to end through the public API with host buffers
     e2e = []
     oh = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
@@ -316,8 +347,10 @@ def run_scope(args, world, rank, local):
                    "head_dim": w.D, "top_p": w.top_p, "online_topk": bool(w.online_topk),
                    "l2": "inputs 2.2 GB >> 126 MB L2, no flush", "parallelism": f"replicas x{world}"},
         "effective_tflops": eff, "plan_ms": plan_ms, "attn_ms": attn_ms, "density": density,
+        "own_dense_ms": dense_ms, "speedup_vs_own_dense": dense_ms / ms_per_call,
         "roofline": {"kernel": "sparse attention (scope_attn)", "bound": "tensor", "achieved": achieved,
-                     "peak": bf16_sus, "unit": "TFLOP/s", "frac": achieved / bf16_sus, "traffic": None,
+                     "peak": bf16_sus, "unit": "TFLOP/s", "frac": achieved / bf16_sus,
+                     "traffic": attn_traffic(w.B * w.H),
                      "peak_source": f"{src} bf16 sustained"},
         "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
