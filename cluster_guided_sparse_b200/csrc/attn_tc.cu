@@ -476,37 +476,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l *= alpha;
                 rescale = true;
             }
-            // p = 2^(s*scale - m) on pairs, reloading S in two 64-column halves;
-            // row sum in two lanes; bf16 pairs written over S.
+            // p = 2^(s*scale - m) on pairs straight from the loaded row; row sum
+            // in four partial lanes; bf16 pairs written over S.
             const float nm = -m_run, sc = a.scale_log2;
             float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                uint32_t q[64];
-                tmem_ld32(tS + h2 * 64, q);
-                tmem_ld32(tS + h2 * 64 + 32, q + 32);
-                tmem_wait_ld();
+            for (int c4 = 0; c4 < BN / 32; ++c4) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int c4 = 0; c4 < 2; ++c4) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int col = h2 * 64 + c4 * 32 + 2 * i;
-                        float x0, x1, p0, p1;
-                        ffma2(x0, x1, __uint_as_float(q[c4 * 32 + 2 * i]), __uint_as_float(q[c4 * 32 + 2 * i + 1]), sc,
-                              sc, nm, nm);
-                        p0 = ex2(x0);
-                        p1 = ex2(x1);
-                        if (valid < BN) {
-                            p0 = col < valid ? p0 : 0.f;
-                            p1 = col + 1 < valid ? p1 : 0.f;
-                        }
-                        if (i & 1) fadd2(lc, ld, p0, p1);
-                        else fadd2(la, lb, p0, p1);
-                        pk[i] = pack_bf16(p0, p1);
-                    }
-                    tmem_st16(tS + h2 * 32 + c4 * 16, pk);
+                for (int i = 0; i < 16; ++i) {
+                    float x0, x1;
+                    ffma2(x0, x1, __uint_as_float(r[c4 * 32 + 2 * i]), __uint_as_float(r[c4 * 32 + 2 * i + 1]), sc, sc,
+                          nm, nm);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    if (i & 1) fadd2(lc, ld, p0, p1);
+                    else fadd2(la, lb, p0, p1);
+                    pk[i] = pack_bf16(p0, p1);
                 }
+                tmem_st16(tS + c4 * 16, pk);
             }
             la += lc;
             lb += ld;
