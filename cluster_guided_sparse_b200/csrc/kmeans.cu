@@ -461,6 +461,14 @@ void launch_km_assign_tiled(const KmProblem &P, int BH, int N, int D, const floa
     count_launches(1);
 }
 
+void km_fixup_launch(const KmProblem &P, int BH, int N, int D, const int32_t *fix_list, const int32_t *fix_count,
+                     cudaStream_t st)
+{
+    (void)BH;
+    km_fixup_kernel<<<148 * 4, 256, 0, st>>>(P, N, D, fix_list, fix_count);
+    count_launches(1);
+}
+
 void launch_km_sort(const KmBatch &b, int BH, int N, cudaStream_t st)
 {
     const int nblk = (N + kSortBlk - 1) / kSortBlk;

@@ -25,6 +25,9 @@ void launch_km_sort(const KmBatch &, int, int, cudaStream_t);
 void launch_bisect(const __nv_bfloat16 *, int, int, int, int, int, int32_t *, int32_t *, double *, int32_t *, float *,
                    float *, int32_t *, int32_t *, int32_t *, cudaStream_t);
 void launch_km_assign_tiled(const KmProblem &, int, int, int, const float *, int32_t *, int32_t *, cudaStream_t);
+cudaError_t km_tc_configure();
+bool launch_km_assign_tc(const KmProblem &, __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, const float *, int32_t *,
+                         int32_t *, int32_t *, cudaStream_t);
 void launch_km_reduce(const KmBatch &, int, int, int, cudaStream_t);
 
 struct SelArgs;
@@ -79,7 +82,7 @@ struct Layout {
     size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
     size_t lut, item_hist, item_id, item_cnt, item_n, r, n, kh, offsets, indices, work, nwork, vb, fix;
-    size_t bis_order, bis_delta;
+    size_t bis_order, bis_delta, q_chi, q_clo;
     size_t total;
 };
 
@@ -224,6 +227,8 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.q_start = take(cur, BH * (L.Cq + 1) * 4);
     L.q_bhist = take(cur, BH * L.Cq * L.nblk * 4);
     L.fix = take(cur, BH * N * 4 + 16);
+    L.q_chi = take(cur, BH * L.Cq * D * 2);
+    L.q_clo = take(cur, BH * L.Cq * D * 2);
     L.bis_order = take(cur, L.bisect ? 2 * BH * N * 4 : 0);
     L.bis_delta = take(cur, L.bisect ? BH * N * 8 : 0);
     L.k_codes = take(cur, 3 * BH * N * 4);
@@ -261,7 +266,7 @@ scope_status check_device(cudaStream_t)
     if (major != 10) return fail(SCOPE_EDEVICE, "libscope.so is built for sm_100a; device has compute capability %d.x", major);
     static bool configured[64] = {false};
     if (dev < 64 && !configured[dev]) {
-        if (km_configure() != cudaSuccess || attn_tc_configure() != cudaSuccess)
+        if (km_configure() != cudaSuccess || attn_tc_configure() != cudaSuccess || km_tc_configure() != cudaSuccess)
             return fail(SCOPE_ECUDA, "kernel attribute setup failed");
         configured[dev] = true;
     }
@@ -395,7 +400,8 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     } else {
     // Key subspaces always, and the queries when they have few clusters, run
     // as one batch on the direct-form kernel; queries with >= 128 clusters use
-    // the register-tiled certified kernel (plus its fp64 fix-up pass).
+    // the certified tensor-core kernel (bf16 hi/lo centroid split, fp64 fix-up
+    // of the rows inside its error margin).
     const bool tiled_q = L.Cq >= 128;
     KmBatch all{};
     for (int i = 0; i < 3; ++i) all.p[i] = key_problem(L, ws, i);
@@ -408,10 +414,13 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     qonly.count = 1;
     int32_t *fix_count = at<int32_t>(ws, L.fix);
     int32_t *fix_list = fix_count + 4;
+    bool tc_ok = true;
     auto assign = [&]() {
         if (tiled_q) {
             launch_km_assign_direct(keys, BH, N, D, s);
-            launch_km_assign_tiled(all.p[3], BH, N, D, at<float>(ws, L.qnorm), fix_list, fix_count, s);
+            tc_ok = tc_ok && launch_km_assign_tc(all.p[3], at<__nv_bfloat16>(ws, L.q_chi), at<__nv_bfloat16>(ws, L.q_clo),
+                                                 BH, N, D, at<float>(ws, L.qnorm), fix_list, fix_count,
+                                                 at<int32_t>(ws, L.stats) + 4, s);
         } else {
             launch_km_assign_direct(all, BH, N, D, s);
         }
@@ -424,6 +433,7 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     }
     assign();
     launch_km_sort(qonly, BH, N, s);
+    if (!tc_ok) return fail(SCOPE_ECUDA, "k-means: tensor map encoding failed");
     }
     if ((st = launch_status("k-means")) != SCOPE_OK) return st;
 
