@@ -17,9 +17,11 @@
 // One CTA = 128 rows (one M=128 tile).  Warps 0-3: argmin epilogue, one row
 // per thread, reading the 128 x 128 score tile of a centroid chunk from TMEM;
 // warp 4: tcgen05.mma issuer and TMEM owner; warp 5: TMA producer (the row
-// tile once, then hi/lo centroid chunks of 128, two stages).  The TMEM
+// tile once, then hi/lo centroid chunks of 128 through one stage).  The TMEM
 // accumulator is double-buffered so chunk c+1's MMAs overlap chunk c's
-// epilogue.
+// epilogue; 96 KB of shared memory and 256 TMEM columns let two CTAs share an
+// SM and hide each other's load latency.  The epilogue keeps eight
+// interleaved (best, arg, second) states so its compare chain is short.
 #include "tcgen05.cuh"
 
 namespace scope {
@@ -39,7 +41,7 @@ struct KtArgs {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kKT, 1)
+__global__ void __launch_bounds__(kKT, 2)
     km_assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmHi,
                         const __grid_constant__ CUtensorMap tmLo, KtArgs a)
 {
@@ -47,7 +49,7 @@ __global__ void __launch_bounds__(kKT, 1)
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     constexpr int TILE = 128 * D * 2;  // one 128-row bf16 tile
     unsigned char *sX = sm;
-    unsigned char *sC = sm + TILE;     // [stage][hi, lo]
+    unsigned char *sC = sm + TILE;     // [hi, lo]
     __shared__ uint64_t bar_x, bar_c_full[2], bar_c_empty[2], bar_acc_full[2], bar_acc_empty[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
@@ -96,10 +98,10 @@ __global__ void __launch_bounds__(kKT, 1)
             for (int cb = 0; cb < D / 64; ++cb)
                 tma_load_2d(smem_u32(sX) + cb * 128 * 128, &tmX, cb * 64, bh * N + p0, &bar_x);
             for (int c = 0; c < nchunks; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !mbar_wait(&bar_c_empty[s], ((c >> 1) - 1) & 1, abort_flag, a.err, 0x40)) break;
+                const int s = 0;
+                if (c >= 1 && !mbar_wait(&bar_c_empty[0], (c - 1) & 1, abort_flag, a.err, 0x40)) break;
                 mbar_expect_tx(&bar_c_full[s], 2 * TILE);
-                const uint32_t dst = smem_u32(sC + s * 2 * TILE);
+                const uint32_t dst = smem_u32(sC);
 #pragma unroll
                 for (int cb = 0; cb < D / 64; ++cb) {
                     tma_load_2d(dst + cb * 128 * 128, &tmHi, cb * 64, bh * C + c * 128, &bar_c_full[s]);
@@ -116,10 +118,10 @@ __global__ void __launch_bounds__(kKT, 1)
             bool ok = mbar_wait(&bar_x, 0, abort_flag, a.err, 0x41);
             for (int c = 0; ok && c < nchunks; ++c) {
                 const int s = c & 1;
-                if (!mbar_wait(&bar_c_full[s], (c >> 1) & 1, abort_flag, a.err, 0x42)) break;
+                if (!mbar_wait(&bar_c_full[0], c & 1, abort_flag, a.err, 0x42)) break;
                 if (c >= 2 && !mbar_wait(&bar_acc_empty[s], ((c >> 1) - 1) & 1, abort_flag, a.err, 0x43)) break;
                 tc_fence_after();
-                const uint32_t ca = smem_u32(sC + s * 2 * TILE);
+                const uint32_t ca = smem_u32(sC);
 #pragma unroll
                 for (int half = 0; half < 2; ++half)
 #pragma unroll
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(kKT, 1)
                                sw128_desc(ca + half * TILE + ko, 16, 1024), idesc, (half > 0 || k > 0));
                     }
                 mma_commit(&bar_acc_full[s]);
-                mma_commit(&bar_c_empty[s]);
+                mma_commit(&bar_c_empty[0]);
             }
         }
         __syncwarp();
@@ -138,8 +140,14 @@ __global__ void __launch_bounds__(kKT, 1)
         const int row = warp * 32 + lane, n = p0 + row;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         float r2 = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-        float b1 = INFINITY, b2 = INFINITY;
-        int a1 = 0;
+        float B1[8], B2[8];
+        int A1[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            B1[q] = INFINITY;
+            B2[q] = INFINITY;
+            A1[q] = 0;
+        }
         bool ok = true;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
@@ -155,20 +163,36 @@ __global__ void __launch_bounds__(kKT, 1)
             tc_fence_before();
             mbar_arrive(&bar_acc_empty[s]);
             const int c0 = c * 128;
+            const float *cnc = cn + c0;
+            const int lim = min(128, C - c0);
 #pragma unroll
             for (int j = 0; j < 128; ++j) {
-                const int cj = c0 + j;
-                if (cj < C) {
-                    const float e = fmaf(-2.f, __uint_as_float(r[j]), __ldg(cn + cj));
-                    if (e < b1) {
-                        b2 = b1;
-                        b1 = e;
-                        a1 = cj;
-                    } else if (e < b2) {
-                        b2 = e;
+                const int q = j & 7;
+                if (j < lim) {
+                    const float e = fmaf(-2.f, __uint_as_float(r[j]), __ldg(cnc + j));
+                    if (e < B1[q]) {
+                        B2[q] = B1[q];
+                        B1[q] = e;
+                        A1[q] = c0 + j;
+                    } else if (e < B2[q]) {
+                        B2[q] = e;
                     }
                 }
             }
+        }
+        // merge the eight states; equal scores keep the lowest centroid index
+        float b1 = B1[0], b2 = B2[0];
+        int a1 = A1[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) {
+            if (B1[q] < b1 || (B1[q] == b1 && A1[q] < a1)) {
+                b2 = fminf(b1, B2[q]);
+                b1 = B1[q];
+                a1 = A1[q];
+            } else {
+                b2 = fminf(b2, B1[q]);
+            }
+            b2 = fminf(b2, B2[q]);
         }
         if (ok && n < N) {
             const float xn = sqrtf(a.xnorm2[(int64_t)bh * N + n]);
@@ -210,10 +234,10 @@ void km_fixup_launch(const KmProblem &P, int BH, int N, int D, const int32_t *fi
 cudaError_t km_tc_configure()
 {
     cudaError_t e = cudaFuncSetAttribute(km_assign_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(5 * 128 * 128 * 2 + 1024));
+                                         (int)(3 * 128 * 128 * 2 + 1024));
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(km_assign_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)(5 * 128 * 64 * 2 + 1024));
+                                (int)(3 * 128 * 64 * 2 + 1024));
 }
 
 // Tensor maps for the rows and the hi/lo centroid tables; false if encoding failed.
@@ -239,9 +263,9 @@ bool launch_km_assign_tc(const KmProblem &P, __nv_bfloat16 *chi, __nv_bfloat16 *
     a.D = D;
     const dim3 grid((N + 127) / 128, BH);
     if (D == 128)
-        km_assign_tc_kernel<128><<<grid, kKT, 5 * 128 * 128 * 2 + 1024, st>>>(tmX, tmHi, tmLo, a);
+        km_assign_tc_kernel<128><<<grid, kKT, 3 * 128 * 128 * 2 + 1024, st>>>(tmX, tmHi, tmLo, a);
     else
-        km_assign_tc_kernel<64><<<grid, kKT, 5 * 128 * 64 * 2 + 1024, st>>>(tmX, tmHi, tmLo, a);
+        km_assign_tc_kernel<64><<<grid, kKT, 3 * 128 * 64 * 2 + 1024, st>>>(tmX, tmHi, tmLo, a);
     count_launches(1);
     km_fixup_launch(P, BH, N, D, fix_list, fix_count, st);
     return true;
