@@ -61,9 +61,34 @@ __global__ void __launch_bounds__(128) km_assign_direct_kernel(KmBatch b, int N,
     const int dn = P.dim_n, C = P.C, T = blockDim.x;
     float *xs = sm;            // [dn][T]
     float *cs = sm + dn * T;   // [dn][CH]
-    for (int idx = threadIdx.x; idx < T * dn; idx += T) {
-        const int r = idx / dn, k = idx % dn, n = n0 + r;
-        xs[k * T + r] = n < N ? __bfloat162float(P.X[((int64_t)bh * N + n) * D + P.dim_off + k]) : 0.f;
+    // rows -> xs[k][r], consecutive threads on consecutive rows so the
+    // transposed stores hit distinct banks; 16-byte loads of 8 dims when the
+    // column range allows it.
+    if (((P.dim_off | dn) & 7) == 0) {
+        for (int idx = threadIdx.x; idx < T * (dn >> 3); idx += T) {
+            const int r = idx % T, k8 = (idx / T) * 8, n = n0 + r;
+            float v[8];
+            if (n < N) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(P.X + ((int64_t)bh * N + n) * D + P.dim_off + k8);
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __bfloat1622float2(h[q]);
+                    v[2 * q] = f.x;
+                    v[2 * q + 1] = f.y;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) v[q] = 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xs[(k8 + q) * T + r] = v[q];
+        }
+    } else {
+        for (int idx = threadIdx.x; idx < T * dn; idx += T) {
+            const int r = idx % T, k = idx / T, n = n0 + r;
+            xs[k * T + r] = n < N ? __bfloat162float(P.X[((int64_t)bh * N + n) * D + P.dim_off + k]) : 0.f;
+        }
     }
     float best = INFINITY;
     int arg = 0;
@@ -71,7 +96,7 @@ __global__ void __launch_bounds__(128) km_assign_direct_kernel(KmBatch b, int N,
     for (int c0 = 0; c0 < C; c0 += CH) {
         __syncthreads();
         for (int idx = threadIdx.x; idx < CH * dn; idx += T) {
-            const int j = idx / dn, k = idx % dn;
+            const int j = idx % CH, k = idx / CH;  // consecutive threads: consecutive centroids
             cs[k * CH + j] = (c0 + j < C) ? cent[(int64_t)(c0 + j) * dn + k] : 0.f;
         }
         __syncthreads();
@@ -393,8 +418,16 @@ __global__ void __launch_bounds__(1024) km_reduce_kernel(KmBatch b, int N, int D
     if (col < dn) {
         const int32_t *perm = P.perm + (int64_t)bh * N + st;
         const __nv_bfloat16 *X = P.X + (int64_t)bh * N * D + P.dim_off + col;
-        for (int m = slice; m < sz; m += slices)
-            acc += __double2ll_rn((double)__bfloat162float(X[(int64_t)perm[m] * D]) * scale);
+        // four members per step so their (perm -> row) load chains overlap
+        int m = slice;
+        for (; m + 3 * slices < sz; m += 4 * slices) {
+            const int i0 = perm[m], i1 = perm[m + slices], i2 = perm[m + 2 * slices], i3 = perm[m + 3 * slices];
+            const float x0 = __bfloat162float(X[(int64_t)i0 * D]), x1 = __bfloat162float(X[(int64_t)i1 * D]);
+            const float x2 = __bfloat162float(X[(int64_t)i2 * D]), x3 = __bfloat162float(X[(int64_t)i3 * D]);
+            acc += __double2ll_rn((double)x0 * scale) + __double2ll_rn((double)x1 * scale) +
+                   __double2ll_rn((double)x2 * scale) + __double2ll_rn((double)x3 * scale);
+        }
+        for (; m < sz; m += slices) acc += __double2ll_rn((double)__bfloat162float(X[(int64_t)perm[m] * D]) * scale);
     }
     part[threadIdx.x] = acc;
     __syncthreads();
