@@ -54,6 +54,7 @@ __global__ void __launch_bounds__(kKT, 2)
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ float red[4];
+    __shared__ __align__(16) float cn_sh[kMaxClusters];
 
     const KmProblem &P = a.P;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -80,7 +81,11 @@ __global__ void __launch_bounds__(kKT, 2)
     // R^2 = max_j ||c_j||^2 (epilogue warps)
     if (warp < 4) {
         float r2 = 0.f;
-        for (int j = threadIdx.x; j < C; j += 128) r2 = fmaxf(r2, cn[j]);
+        for (int j = threadIdx.x; j < (C + 127) / 128 * 128; j += 128) {
+            const float v = j < C ? cn[j] : 0.f;
+            cn_sh[j] = j < C ? v : __int_as_float(0x7f800000);  // padding never wins
+            r2 = fmaxf(r2, v);
+        }
         r2 = warp_max(r2);
         if (lane == 0) red[warp] = r2;
     }
@@ -163,21 +168,18 @@ __global__ void __launch_bounds__(kKT, 2)
             tc_fence_before();
             mbar_arrive(&bar_acc_empty[s]);
             const int c0 = c * 128;
-            const float *cnc = cn + c0;
-            const int lim = min(128, C - c0);
+            const float4 *cnc = reinterpret_cast<const float4 *>(cn_sh + c0);
 #pragma unroll
             for (int j = 0; j < 128; ++j) {
                 const int q = j & 7;
-                if (j < lim) {
-                    const float e = fmaf(-2.f, __uint_as_float(r[j]), __ldg(cnc + j));
-                    if (e < B1[q]) {
-                        B2[q] = B1[q];
-                        B1[q] = e;
-                        A1[q] = c0 + j;
-                    } else if (e < B2[q]) {
-                        B2[q] = e;
-                    }
-                }
+                const float4 c4 = cnc[j >> 2];
+                const float cj = (j & 3) == 0 ? c4.x : (j & 3) == 1 ? c4.y : (j & 3) == 2 ? c4.z : c4.w;
+                const float e = fmaf(-2.f, __uint_as_float(r[j]), cj);
+                // branch-free best / second-best update; an equal score keeps the
+                // earlier (lower) index and collapses the margin to zero
+                B2[q] = fminf(B2[q], fmaxf(B1[q], e));
+                A1[q] = e < B1[q] ? c0 + j : A1[q];
+                B1[q] = fminf(B1[q], e);
             }
         }
         // merge the eight states; equal scores keep the lowest centroid index
