@@ -29,6 +29,7 @@ struct KmProblem {
     int32_t *perm;              // [BH][N]   members cluster by cluster, ascending
     int32_t *start;             // [BH][C+1] cluster starts in perm
     int32_t *blockhist;         // [BH][C][nblk]
+    unsigned long long *sums;   // [BH][C][dim_n] fixed-point member sums, zero between updates (or null)
 };
 
 struct KmBatch {

@@ -45,86 +45,133 @@ __global__ void km_init_kernel(KmBatch b, int N, int D, uint32_t seed)
     }
 }
 
-// -------------------------------------------------------------- assign (direct form)
-// One thread per row; the CTA's rows are staged transposed in shared memory
-// and centroids stream through in chunks of CH, transposed so one 16-byte
-// broadcast load feeds four centroids.  d = sum_k (x_k - c_k)^2 in fp32: no
-// cancellation, relative error <= (dim+2) * 2^-24 of the distance.
-template <int CH>
-__global__ void __launch_bounds__(128) km_assign_direct_kernel(KmBatch b, int N, int D)
+// Packed f32x2 arithmetic on 64-bit register pairs (lane 0 = low word), IEEE
+// round-to-nearest without flushing subnormals: each lane gives the same fp32
+// result as the scalar instruction.
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi)
 {
-    extern __shared__ __align__(16) float sm[];
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void unpack2(unsigned long long v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// acc + d * d
+__device__ __forceinline__ unsigned long long sqacc2(unsigned long long acc, unsigned long long d)
+{
+    asm("fma.rn.f32x2 %0, %1, %1, %0;" : "+l"(acc) : "l"(d));
+    return acc;
+}
+
+// -------------------------------------------------------------- assign (direct form)
+// Two adjacent rows per thread (256 per CTA).  Their columns are staged in
+// shared memory as bf16 pairs (one 32-bit word per column, transposed so
+// consecutive threads read consecutive words); the centroids stream through in
+// chunks of W, negated and duplicated ((-c, -c) per column), so one packed add
+// forms x - c for both rows and one packed FMA adds both squares: the pair
+// (x0, x1) is built once per column and every 16-byte broadcast load feeds two
+// centroids x two rows.  d = sum_k (x_k - c_k)^2 in fp32 with k ascending: no
+// cancellation, relative error <= (dim+2) * 2^-24 of the distance.
+constexpr int kDirRows = 256, kDirCH = 32;
+
+template <int W>
+__device__ __forceinline__ void direct_chunk(const uint32_t *xs, const unsigned long long *cs, int dn, int c0, int C,
+                                             float (&best)[2], int (&arg)[2])
+{
+    unsigned long long acc[W];
+#pragma unroll
+    for (int j = 0; j < W; ++j) acc[j] = 0ull;
+    for (int k = 0; k < dn; ++k) {
+        const uint32_t xp = xs[k * (kDirRows / 2) + threadIdx.x];
+        const unsigned long long x = pack2(__uint_as_float(xp << 16), __uint_as_float(xp & 0xffff0000u));
+        const ulonglong2 *c2 = reinterpret_cast<const ulonglong2 *>(cs + k * kDirCH);
+#pragma unroll
+        for (int j2 = 0; j2 < W / 2; ++j2) {
+            const ulonglong2 c = c2[j2];
+            acc[2 * j2] = sqacc2(acc[2 * j2], add2(x, c.x));
+            acc[2 * j2 + 1] = sqacc2(acc[2 * j2 + 1], add2(x, c.y));
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+        float d0, d1;
+        unpack2(acc[j], d0, d1);
+        const bool in = c0 + j < C;
+        const bool lt0 = in && d0 < best[0], lt1 = in && d1 < best[1];  // first minimum wins
+        best[0] = lt0 ? d0 : best[0];
+        arg[0] = lt0 ? c0 + j : arg[0];
+        best[1] = lt1 ? d1 : best[1];
+        arg[1] = lt1 ? c0 + j : arg[1];
+    }
+}
+
+__global__ void __launch_bounds__(kDirRows / 2) km_assign_direct_kernel(KmBatch b, int N, int D)
+{
+    extern __shared__ __align__(16) uint32_t smw[];
     const KmProblem &P = b.p[blockIdx.z];
-    const int bh = blockIdx.y;
-    const int n0 = blockIdx.x * blockDim.x;
+    const int bh = blockIdx.y, T = kDirRows / 2;
+    const int n0 = blockIdx.x * kDirRows;
     if (n0 >= N) return;
-    const int dn = P.dim_n, C = P.C, T = blockDim.x;
-    float *xs = sm;            // [dn][T]
-    float *cs = sm + dn * T;   // [dn][CH]
-    // rows -> xs[k][r], consecutive threads on consecutive rows so the
-    // transposed stores hit distinct banks; 16-byte loads of 8 dims when the
-    // column range allows it.
+    const int dn = P.dim_n, C = P.C;
+    uint32_t *xs = smw;                                                          // [dn][T]
+    unsigned long long *cs = reinterpret_cast<unsigned long long *>(smw + ((dn * T + 3) & ~3));  // [dn][kDirCH]
+    const __nv_bfloat16 *Xb = P.X + (int64_t)bh * N * D + P.dim_off;
+    // row pair t -> xs[k][t] = bf16(row 2t) | bf16(row 2t+1) << 16
     if (((P.dim_off | dn) & 7) == 0) {
         for (int idx = threadIdx.x; idx < T * (dn >> 3); idx += T) {
-            const int r = idx % T, k8 = (idx / T) * 8, n = n0 + r;
-            float v[8];
-            if (n < N) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(P.X + ((int64_t)bh * N + n) * D + P.dim_off + k8);
-                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+            const int t = idx % T, k8 = (idx / T) * 8, n = n0 + 2 * t;
+            uint4 u0 = make_uint4(0u, 0u, 0u, 0u), u1 = u0;
+            if (n < N) u0 = *reinterpret_cast<const uint4 *>(Xb + (int64_t)n * D + k8);
+            if (n + 1 < N) u1 = *reinterpret_cast<const uint4 *>(Xb + (int64_t)(n + 1) * D + k8);
+            const uint32_t a[4] = {u0.x, u0.y, u0.z, u0.w}, c[4] = {u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 f = __bfloat1622float2(h[q]);
-                    v[2 * q] = f.x;
-                    v[2 * q + 1] = f.y;
-                }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) v[q] = 0.f;
+            for (int q = 0; q < 4; ++q) {
+                xs[(k8 + 2 * q) * T + t] = __byte_perm(a[q], c[q], 0x5410);
+                xs[(k8 + 2 * q + 1) * T + t] = __byte_perm(a[q], c[q], 0x7632);
             }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) xs[(k8 + q) * T + r] = v[q];
         }
     } else {
+        const unsigned short *Xs = reinterpret_cast<const unsigned short *>(Xb);
         for (int idx = threadIdx.x; idx < T * dn; idx += T) {
-            const int r = idx % T, k = idx / T, n = n0 + r;
-            xs[k * T + r] = n < N ? __bfloat162float(P.X[((int64_t)bh * N + n) * D + P.dim_off + k]) : 0.f;
+            const int t = idx % T, k = idx / T, n = n0 + 2 * t;
+            const uint32_t lo = n < N ? Xs[(int64_t)n * D + k] : 0u;
+            const uint32_t hi = n + 1 < N ? Xs[(int64_t)(n + 1) * D + k] : 0u;
+            xs[k * T + t] = lo | (hi << 16);
         }
     }
-    float best = INFINITY;
-    int arg = 0;
+    float best[2] = {INFINITY, INFINITY};
+    int arg[2] = {0, 0};
     const float *cent = P.cent + (int64_t)bh * C * dn;
-    for (int c0 = 0; c0 < C; c0 += CH) {
+    for (int c0 = 0; c0 < C; c0 += kDirCH) {
         __syncthreads();
-        for (int idx = threadIdx.x; idx < CH * dn; idx += T) {
-            const int j = idx % CH, k = idx / CH;  // consecutive threads: consecutive centroids
-            cs[k * CH + j] = (c0 + j < C) ? cent[(int64_t)(c0 + j) * dn + k] : 0.f;
+        for (int idx = threadIdx.x; idx < kDirCH * dn; idx += T) {
+            const int j = idx % kDirCH, k = idx / kDirCH;  // consecutive threads: consecutive centroids
+            const float v = (c0 + j < C) ? -cent[(int64_t)(c0 + j) * dn + k] : 0.f;
+            cs[k * kDirCH + j] = pack2(v, v);
         }
         __syncthreads();
-        float acc[CH];
-#pragma unroll
-        for (int j = 0; j < CH; ++j) acc[j] = 0.f;
-        for (int k = 0; k < dn; ++k) {
-            const float xv = xs[k * T + threadIdx.x];
-            const float4 *c4 = reinterpret_cast<const float4 *>(cs + k * CH);
-#pragma unroll
-            for (int j4 = 0; j4 < CH / 4; ++j4) {
-                const float4 c = c4[j4];
-                float d;
-                d = xv - c.x; acc[4 * j4 + 0] = fmaf(d, d, acc[4 * j4 + 0]);
-                d = xv - c.y; acc[4 * j4 + 1] = fmaf(d, d, acc[4 * j4 + 1]);
-                d = xv - c.z; acc[4 * j4 + 2] = fmaf(d, d, acc[4 * j4 + 2]);
-                d = xv - c.w; acc[4 * j4 + 3] = fmaf(d, d, acc[4 * j4 + 3]);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < CH; ++j)
-            if (c0 + j < C && acc[j] < best) {
-                best = acc[j];
-                arg = c0 + j;
-            }
+        if (C - c0 <= 16) direct_chunk<16>(xs, cs, dn, c0, C, best, arg);
+        else direct_chunk<kDirCH>(xs, cs, dn, c0, C, best, arg);
     }
-    const int n = n0 + threadIdx.x;
-    if (n < N) P.labels[(int64_t)bh * N + n] = arg;
+    const int n = n0 + 2 * threadIdx.x;
+    if (n < N) P.labels[(int64_t)bh * N + n] = arg[0];
+    if (n + 1 < N) P.labels[(int64_t)bh * N + n + 1] = arg[1];
+}
+
+static size_t direct_smem(int dn)
+{
+    return (size_t)((dn * (kDirRows / 2) + 3) & ~3) * 4 + (size_t)dn * kDirCH * 8;
 }
 
 // -------------------------------------------------------------- assign (tiled, certified)
@@ -445,6 +492,127 @@ __global__ void __launch_bounds__(1024) km_reduce_kernel(KmBatch b, int N, int D
     }
 }
 
+// -------------------------------------------------------------- update (segmented)
+// The same fixed-point sums, accumulated over the sorted member order in
+// equal segments instead of one CTA per cluster, so a cluster of 7000 keys
+// no longer runs as one long chain of dependent loads.  Each warp owns 128
+// consecutive sorted positions; a row is read by ceil(dim_n/4) lanes with one
+// 8-byte load each (several rows per warp step when dim_n is small), and a
+// lane keeps int64 sums of its four columns until its rows cross into the next
+// cluster, when it adds them to the cluster's sums with integer atomics.
+// Integer addition is associative, so the totals (and the means) do not
+// depend on the order in which segments arrive.  x * 2^S is exact in fp32
+// (bf16 input, S in [0, 40]), so its rounding to an integer equals the fp64
+// form of the per-cluster kernel above.
+constexpr int kSegWarps = 8, kSegRows = 128, kSegUnroll = 16;
+
+__global__ void __launch_bounds__(kSegWarps * 32, 3) km_accum_kernel(KmBatch b, int N, int D)
+{
+    __shared__ int32_t rows_sh[kSegWarps][kSegRows];
+    const KmProblem &P = b.p[blockIdx.z];
+    const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int p0 = (blockIdx.x * kSegWarps + warp) * kSegRows;
+    if (p0 >= N) return;
+    const int p1 = min(N, p0 + kSegRows);
+    const int dn = P.dim_n, C = P.C, quads = (dn + 3) >> 2;
+    int lanes = 1;
+    while (lanes < quads) lanes <<= 1;
+    const int R = 32 / lanes, slot = lane / lanes, d0 = 4 * (lane % lanes);
+    const int nv = d0 < dn ? min(4, dn - d0) : 0;
+    const bool vec = nv == 4 && ((P.dim_off & 3) == 0);
+    const int32_t *start = P.start + (int64_t)bh * (C + 1);
+    const int32_t *perm = P.perm + (int64_t)bh * N;
+    const __nv_bfloat16 *X = P.X + (int64_t)bh * N * D + P.dim_off + d0;
+    unsigned long long *sums = P.sums + (int64_t)bh * C * dn + d0;
+    const float scale = ldexpf(1.f, fixed_shift(P.maxabs, N));
+    // the warp's member rows, read once and coalesced
+    int32_t *rows = rows_sh[warp];
+    for (int t = lane; t < kSegRows; t += 32) rows[t] = p0 + t < p1 ? perm[p0 + t] : 0;
+    __syncwarp();
+
+    int p = p0 + slot;
+    if (p >= p1) return;
+    // cluster of position p: the last c with start[c] <= p (skips empty ones)
+    int lo = 0, hi = C;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (start[mid] <= p) lo = mid;
+        else hi = mid;
+    }
+    int cur = lo, nxt = start[cur + 1];
+    long long acc[4] = {0, 0, 0, 0};
+    bool any = false;
+    for (; p < p1; p += kSegUnroll * R) {
+        uint2 raw[kSegUnroll];
+#pragma unroll
+        for (int u = 0; u < kSegUnroll; ++u) {
+            raw[u] = make_uint2(0u, 0u);
+            if (p + u * R < p1) {
+                const __nv_bfloat16 *x = X + (int64_t)rows[p + u * R - p0] * D;
+                if (vec) {
+                    raw[u] = *reinterpret_cast<const uint2 *>(x);
+                } else if (nv > 0) {
+                    const unsigned short *xs = reinterpret_cast<const unsigned short *>(x);
+                    const uint32_t h0 = xs[0], h1 = nv > 1 ? xs[1] : 0u, h2 = nv > 2 ? xs[2] : 0u,
+                                   h3 = nv > 3 ? xs[3] : 0u;
+                    raw[u] = make_uint2(h0 | (h1 << 16), h2 | (h3 << 16));
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kSegUnroll; ++u) {
+            const int pu = p + u * R;
+            if (pu < p1) {
+                while (pu >= nxt) {
+                    if (any)
+                        for (int i = 0; i < nv; ++i) atomicAdd(sums + (int64_t)cur * dn + i, (unsigned long long)acc[i]);
+                    acc[0] = acc[1] = acc[2] = acc[3] = 0;
+                    any = false;
+                    ++cur;
+                    nxt = start[cur + 1];
+                }
+                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw[u].x));
+                const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw[u].y));
+                acc[0] += __float2ll_rn(a.x * scale);
+                acc[1] += __float2ll_rn(a.y * scale);
+                acc[2] += __float2ll_rn(c.x * scale);
+                acc[3] += __float2ll_rn(c.y * scale);
+                any = true;
+            }
+        }
+    }
+    if (any)
+        for (int i = 0; i < nv; ++i) atomicAdd(sums + (int64_t)cur * dn + i, (unsigned long long)acc[i]);
+}
+
+// Means from the segmented sums (same rounding as km_reduce_kernel), squared
+// norms, and the sums cleared for the next update.
+__global__ void __launch_bounds__(128) km_finalize_kernel(KmBatch b, int N)
+{
+    __shared__ float cs[128];
+    const KmProblem &P = b.p[blockIdx.z];
+    const int c = blockIdx.x, bh = blockIdx.y, d = threadIdx.x;
+    if (c >= P.C) return;
+    const int dn = P.dim_n;
+    const int32_t *start = P.start + (int64_t)bh * (P.C + 1);
+    const int sz = start[c + 1] - start[c];
+    const double scale = ldexp(1.0, fixed_shift(P.maxabs, N));
+    unsigned long long *sums = P.sums + ((int64_t)bh * P.C + c) * dn;
+    float *cent = P.cent + ((int64_t)bh * P.C + c) * dn;
+    if (d < dn) {
+        const long long s = (long long)sums[d];
+        sums[d] = 0ull;
+        if (sz > 0) cent[d] = (float)((double)s / scale / (double)sz);
+        cs[d] = cent[d];
+    }
+    __syncthreads();
+    if (d == 0) {
+        float s = 0.f;
+        for (int k = 0; k < dn; ++k) s = fmaf(cs[k], cs[k], s);
+        P.cn[(int64_t)bh * P.C + c] = s;
+    }
+}
+
 // -------------------------------------------------------------- launchers
 static int max_C(const KmBatch &b)
 {
@@ -462,8 +630,8 @@ static int max_dim(const KmBatch &b)
 
 cudaError_t km_configure()
 {
-    cudaError_t e = cudaFuncSetAttribute(km_assign_direct_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (128 + 32) * 128 * 4);
+    cudaError_t e = cudaFuncSetAttribute(km_assign_direct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)direct_smem(128));
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(km_assign_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (128 * kTP + kKS * kTC) * (int)sizeof(float));
@@ -477,9 +645,8 @@ void launch_km_init(const KmBatch &b, int BH, int N, int D, uint32_t seed, cudaS
 
 void launch_km_assign_direct(const KmBatch &b, int BH, int N, int D, cudaStream_t st)
 {
-    const int dn = max_dim(b);
-    const size_t smem = (size_t)(128 + 32) * dn * sizeof(float);
-    km_assign_direct_kernel<32><<<dim3((N + 127) / 128, BH, b.count), 128, smem, st>>>(b, N, D);
+    km_assign_direct_kernel<<<dim3((N + kDirRows - 1) / kDirRows, BH, b.count), kDirRows / 2,
+                              direct_smem(max_dim(b)), st>>>(b, N, D);
     count_launches(1);
 }
 
@@ -514,8 +681,17 @@ void launch_km_sort(const KmBatch &b, int BH, int N, cudaStream_t st)
     count_launches(1);
 }
 
+// With sums buffers (every problem of the batch has one): segmented
+// accumulation + finalize; without: one CTA per cluster.
 void launch_km_reduce(const KmBatch &b, int BH, int N, int D, cudaStream_t st)
 {
+    if (b.p[0].sums) {
+        const int per_cta = kSegWarps * kSegRows;
+        km_accum_kernel<<<dim3((N + per_cta - 1) / per_cta, BH, b.count), kSegWarps * 32, 0, st>>>(b, N, D);
+        km_finalize_kernel<<<dim3(max_C(b), BH, b.count), 128, 0, st>>>(b, N);
+        count_launches(2);
+        return;
+    }
     km_reduce_kernel<<<dim3(max_C(b), BH, b.count), 1024, 0, st>>>(b, N, D);
     count_launches(1);
 }

@@ -82,7 +82,7 @@ struct Layout {
     size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
     size_t lut, item_hist, item_id, item_cnt, item_n, r, n, kh, offsets, indices, work, nwork, vb, fix;
-    size_t bis_order, bis_delta, q_chi, q_clo;
+    size_t bis_order, bis_delta, q_chi, q_clo, q_sums, k_sums[3], sums_bytes;
     size_t total;
 };
 
@@ -229,6 +229,13 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.fix = take(cur, BH * N * 4 + 16);
     L.q_chi = take(cur, BH * L.Cq * D * 2);
     L.q_clo = take(cur, BH * L.Cq * D * 2);
+    {
+        // fixed-point centroid sums of every k-means problem, one zeroed region
+        const size_t s0 = cur;
+        L.q_sums = take(cur, BH * L.Cq * D * 8);
+        for (int i = 0; i < 3; ++i) L.k_sums[i] = take(cur, BH * L.C[i] * (L.ds[i] > 0 ? L.ds[i] : 1) * 8);
+        L.sums_bytes = cur - s0;
+    }
     L.bis_order = take(cur, L.bisect ? 2 * BH * N * 4 : 0);
     L.bis_delta = take(cur, L.bisect ? BH * N * 8 : 0);
     L.k_codes = take(cur, 3 * BH * N * 4);
@@ -339,6 +346,7 @@ static KmProblem key_problem(const Layout &L, char *ws, int s)
     P.perm = at<int32_t>(ws, L.k_perm[s]);
     P.start = at<int32_t>(ws, L.k_start[s]);
     P.blockhist = at<int32_t>(ws, L.k_bhist[s]);
+    P.sums = at<unsigned long long>(ws, L.k_sums[s]);
     return P;
 }
 
@@ -357,6 +365,7 @@ static KmProblem query_problem(const Layout &L, char *ws)
     P.perm = at<int32_t>(ws, L.q_perm);
     P.start = at<int32_t>(ws, L.q_start);
     P.blockhist = at<int32_t>(ws, L.q_bhist);
+    P.sums = at<unsigned long long>(ws, L.q_sums);
     return P;
 }
 
@@ -425,6 +434,7 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
             launch_km_assign_direct(all, BH, N, D, s);
         }
     };
+    cudaMemsetAsync(ws + L.q_sums, 0, L.sums_bytes, s);
     launch_km_init(all, BH, N, D, p->init_seed, s);
     for (int it = 0; it < p->iters; ++it) {
         assign();
