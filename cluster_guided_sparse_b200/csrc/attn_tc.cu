@@ -6,10 +6,12 @@
 // of 128 keys.  Both Q tiles share every gathered K/V tile, which halves the
 // K/V bytes per flop (the tiles come from L2: a head's K/V is 61 MB at 720p).
 //
-// Warp roles (352 threads):
+// Warp roles (384 threads; warp w runs on SM sub-partition w % 4, so each
+// sub-partition hosts two softmax warps and at most one other busy warp):
 //   warps 0-3  softmax / epilogue of Q tile 0 (one thread per query row)
 //   warps 4-7  softmax / epilogue of Q tile 1
-//   warp 8     tcgen05.mma issuer (one lane), owns the TMEM allocation
+//   warp 8     idle (keeps the issuer off sub-partition 0)
+//   warp 11    tcgen05.mma issuer (one lane), owns the TMEM allocation
 //   warps 9-10 producer: Q rows and the listed K and V rows by coalesced
 //              16-byte cp.async (16 lanes per 256-byte row) into 128B-swizzled
 //              shared-memory tiles, 2 stages each; K and V have their own
@@ -39,7 +41,8 @@ namespace scope {
 
 namespace tc {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
+constexpr int kMmaWarp = 11;
 constexpr int BN = 128;       // keys per K/V tile
 constexpr int BM = 128;       // rows per Q tile
 
@@ -96,20 +99,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ntiles = (nk + BN - 1) / BN;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bar_q, 64);
+        // producer and softmax barriers take one arrival per warp (lane 0,
+        // after the warp's own waits, fences and a __syncwarp)
+        mbar_init(&bar_q, 2);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bar_k_full[i], 64);
+            mbar_init(&bar_k_full[i], 2);
             mbar_init(&bar_k_empty[i], 1);
-            mbar_init(&bar_v_full[i], 64);
+            mbar_init(&bar_v_full[i], 2);
             mbar_init(&bar_v_empty[i], 1);
             mbar_init(&bar_s_full[i], 1);
-            mbar_init(&bar_p_full[i], 128);
+            mbar_init(&bar_p_full[i], 4);
             mbar_init(&bar_o_final[i], 1);
         }
         abort_sh = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&tmem_base_sh)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
@@ -119,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = tmem_base_sh;
     volatile int *abort_flag = &abort_sh;
 
-    if (warp >= 9) {
+    if (warp == 9 || warp == 10) {
         // ------------------------------------------------------------ producer
         // 64 threads; a warp instruction covers 32 / (D/8) whole rows, so
         // every 16-byte chunk request is part of a fully used 128-byte line.
@@ -136,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         cp_async_commit();
         cp_async_wait_all();
         fence_async_smem();
-        mbar_arrive(&bar_q);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_q);
         // Rows past the list repeat the last listed key (finite V, masked P).
         // A tile's keys are read once, up front (independent loads), and
         // serve both its K and its V rows.
@@ -164,7 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // in flight: K(j), V(j)
             cp_async_wait1();
             fence_async_smem();
-            mbar_arrive(&bar_k_full[j & 1]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_k_full[j & 1]);
             if (more) {
                 load_keys(j + 1);
                 if (j + 1 >= 2 && !mbar_wait(&bar_k_empty[(j + 1) & 1], (((j + 1) >> 1) - 1) & 1, abort_flag, a.err,
@@ -176,7 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cp_async_wait_all();
             }
             fence_async_smem();
-            mbar_arrive(&bar_v_full[j & 1]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_v_full[j & 1]);
             if (more) {
                 if (j + 1 >= 2 && !mbar_wait(&bar_v_empty[(j + 1) & 1], (((j + 1) >> 1) - 1) & 1, abort_flag, a.err,
                                              0x11))
@@ -185,21 +193,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         cp_async_wait_all();
-    } else if (warp == 8) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16(BN, false);
             const uint32_t id_pv = idesc_bf16(D, true);
-            const uint32_t sQa = smem_u32(sQ);
             const int nt = two ? 2 : 1;
+            // descriptors of the first tile / stage; the start-address field
+            // (bits 0-13, 16-byte units) takes the offsets as plain adds
+            const uint64_t dq = sw128_desc(smem_u32(sQ), 16, 1024);
+            const uint64_t dk = sw128_desc(smem_u32(sK), 16, 1024);
+            const uint64_t dv = sw128_desc(smem_u32(sV), BN * 128, 1024);
             auto issue_qk = [&](int t, int j) {
-                const uint32_t sKa = smem_u32(sK + (j & 1) * KV_BYTES);
+                const uint64_t aq = dq + (uint64_t)((t * QT_BYTES) >> 4);
+                const uint64_t bk = dk + (uint64_t)(((j & 1) * KV_BYTES) >> 4);
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t ko = (k >> 2) * (BM * 128) + (k & 3) * 32;
-                    mma_ss(tmem + t * 128, sw128_desc(sQa + t * QT_BYTES + ko, 16, 1024),
-                           sw128_desc(sKa + (k >> 2) * (BN * 128) + (k & 3) * 32, 16, 1024), id_qk, k > 0);
-                }
+                for (int k = 0; k < D / 16; ++k)
+                    mma_ss(tmem + t * 128, aq + (uint64_t)(((k >> 2) * (BM * 128) + (k & 3) * 32) >> 4),
+                           bk + (uint64_t)(((k >> 2) * (BN * 128) + (k & 3) * 32) >> 4), id_qk, k > 0);
                 mma_commit(&bar_s_full[t]);
                 if (t == nt - 1) mma_commit(&bar_k_empty[j & 1]);
             };
@@ -212,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int s = j & 1;
                 if (!mbar_wait(&bar_v_full[s], (j >> 1) & 1, abort_flag, a.err, 0x24)) break;
-                const uint32_t sVa = smem_u32(sV + s * KV_BYTES);
+                const uint64_t bv = dv + (uint64_t)((s * KV_BYTES) >> 4);
                 for (int t = 0; t < nt; ++t) {
                     if (!mbar_wait(&bar_p_full[t], j & 1, abort_flag, a.err, 0x22)) {
                         ok = false;
@@ -221,8 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < BN / 16; ++k)
-                        mma_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8,
-                               sw128_desc(sVa + k * 2048, BN * 128, 1024), id_pv, (j > 0 || k > 0));
+                        mma_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, bv + (uint64_t)((k * 2048) >> 4), id_pv,
+                               (j > 0 || k > 0));
                     if (t == nt - 1) mma_commit(&bar_v_empty[s]);
                     if (j + 1 < ntiles) {
                         if (t == 0 && !mbar_wait(&bar_k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.err,
@@ -238,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp < 8) {
         // ------------------------------------------------------------ softmax + epilogue
         const int t = warp >> 2;           // Q tile of this warpgroup
         const int wq = warp & 3;           // TMEM lane quarter
@@ -265,13 +276,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < BN; ++i)
                     if (i >= valid) r[i] = __float_as_uint(-INFINITY);
             }
-            float m8[8];
+            // row max: three-input max, two new values per instruction, four chains
+            float m4[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) m8[i] = __uint_as_float(r[i]);
+            for (int i = 0; i < 4; ++i) m4[i] = __uint_as_float(r[i]);
 #pragma unroll
-            for (int i = 8; i < BN; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(r[i]));
-            const float mraw = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            for (int i = 4; i < BN; i += 2)
+                m4[(i >> 1) & 3] = fmax3(m4[(i >> 1) & 3], __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+            const float mraw = fmax3(fmax3(m4[0], m4[1], m4[2]), m4[3], m4[3]);
             const float mt = mraw * a.scale_log2;
             // Lazy rescale: move the reference max only when it grew by > 8
             // (log2 units); O and l are scaled after P is written, so the S
@@ -289,23 +301,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // p = 2^(s*scale - m) on pairs straight from the loaded row; row sum
             // in four partial lanes; bf16 pairs written over S.
-            const float nm = -m_run, sc = a.scale_log2;
-            float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
+            const uint64_t scp = f2pack(a.scale_log2, a.scale_log2), nmp = f2pack(-m_run, -m_run);
+            uint64_t sA = 0ull, sB = 0ull;  // (0.f, 0.f)
 #pragma unroll
             for (int c4 = 0; c4 < BN / 32; ++c4) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
+                    const uint64_t x2 = ffma2(
+                        f2pack(__uint_as_float(r[c4 * 32 + 2 * i]), __uint_as_float(r[c4 * 32 + 2 * i + 1])), scp, nmp);
                     float x0, x1;
-                    ffma2(x0, x1, __uint_as_float(r[c4 * 32 + 2 * i]), __uint_as_float(r[c4 * 32 + 2 * i + 1]), sc, sc,
-                          nm, nm);
+                    f2unpack(x2, x0, x1);
                     const float p0 = ex2(x0), p1 = ex2(x1);
-                    if (i & 1) fadd2(lc, ld, p0, p1);
-                    else fadd2(la, lb, p0, p1);
+                    if (i & 1) sB = fadd2(sB, f2pack(p0, p1));
+                    else sA = fadd2(sA, f2pack(p0, p1));
                     pk[i] = pack_bf16(p0, p1);
                 }
                 tmem_st16(tS + c4 * 16, pk);
             }
+            float la, lb, lc, ld;
+            f2unpack(sA, la, lb);
+            f2unpack(sB, lc, ld);
             la += lc;
             lb += ld;
             l += la + lb;
@@ -322,7 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bar_p_full[t]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_p_full[t]);
         }
         if (ok && mbar_wait(&bar_o_final[t], 0, abort_flag, a.err, 0x38 + t)) {
             tc_fence_after();
@@ -352,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
     }
