@@ -174,168 +174,9 @@ static size_t direct_smem(int dn)
     return (size_t)((dn * (kDirRows / 2) + 3) & ~3) * 4 + (size_t)dn * kDirCH * 8;
 }
 
-// -------------------------------------------------------------- assign (tiled, certified)
-// Query assignment for C >= 128: each CTA scores 128 rows against all
-// centroids in 128-wide chunks with 8x8 register tiles per thread, using the
-// expanded form e_j = ||c_j||^2 - 2 x.c_j (one FMA per row-centroid-dim).
-// The fp32 error of every e_j is at most
-//   B = (dim + 2) * 2^-24 * (2 |x| R + R^2),   R = max_j |c_j|
-// (dot-product and norm rounding bounds), so if the runner-up beats the best
-// by more than 2B the argmin is certain; rows inside the margin (and exact
-// ties) are listed and re-decided by km_fixup_kernel in fp64 on the direct
-// form.  The labels are thus those of exact arithmetic on the stored fp32
-// centroids and bf16 rows.
-constexpr int kTP = 128, kTC = 128, kKS = 32;
-
-__device__ __forceinline__ void better(float &b1, int &a1, float &b2, float e, int j)
-{
-    if (e < b1 || (e == b1 && j < a1)) {
-        b2 = b1;
-        b1 = e;
-        a1 = j;
-    } else if (e < b2) {
-        b2 = e;
-    }
-}
-
-// Layout: the CTA's 128 rows stay in shared memory for all dims (fp32,
-// transposed [dim][row]); centroid slices of 32 dims x 128 centroids are
-// prefetched into registers while the previous slice is consumed.  Thread
-// (ty, tx) owns rows 8ty..8ty+7 and centroids {4tx..4tx+3, 64+4tx..64+4tx+3},
-// so a half-warp's 16-byte centroid loads are contiguous (no bank conflict).
-__global__ void __launch_bounds__(256, 2) km_assign_tiled_kernel(KmProblem P, int N, int D, const float *xnorm2,
-                                                                 int32_t *fix_list, int32_t *fix_count)
-{
-    extern __shared__ __align__(16) float smt[];
-    const int dn = P.dim_n;
-    float *xs = smt;              // [dn][kTP]
-    float *cs = smt + dn * kTP;   // [kKS][kTC]
-    __shared__ float red[8];
-    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-    const int bh = blockIdx.y, p0 = blockIdx.x * kTP;
-    const int C = P.C;
-    const __nv_bfloat16 *X = P.X + (int64_t)bh * N * D + P.dim_off;
-    const float *cent = P.cent + (int64_t)bh * C * dn;
-    const float *cn = P.cn + (int64_t)bh * C;
-
-    float r2 = 0.f;
-    for (int j = tid; j < C; j += 256) r2 = fmaxf(r2, cn[j]);
-    r2 = warp_max(r2);
-    if ((tid & 31) == 0) red[tid >> 5] = r2;
-    // rows, once: consecutive lanes take consecutive rows (conflict-free stores)
-    for (int idx = tid; idx < kTP * (dn / 8); idx += 256) {
-        const int p = idx & (kTP - 1), k8 = (idx >> 7) * 8, n = p0 + p;
-        float v[8];
-        if (n < N) {
-            const uint4 u = *reinterpret_cast<const uint4 *>(X + (int64_t)n * D + k8);
-            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float2 f = __bfloat1622float2(h[q]);
-                v[2 * q] = f.x;
-                v[2 * q + 1] = f.y;
-            }
-        } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) v[q] = 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) xs[(k8 + q) * kTP + p] = v[q];
-    }
-    __syncthreads();
-    r2 = red[0];
-    for (int i = 1; i < 8; ++i) r2 = fmaxf(r2, red[i]);
-
-    // running (best, arg, second) of row 8ty+tx, kept by lane tx < 8
-    float rb1 = INFINITY, rb2 = INFINITY;
-    int ra1 = 0;
-    const int nslices = dn / kKS;
-    // centroid slice (c0, k0) -> registers: 4 float4 per thread
-    float4 pre[4];
-    auto fetch = [&](int c0, int k0) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int idx = tid + q * 256, c = idx & (kTC - 1), k4 = (idx >> 7) * 4;
-            pre[q] = (c0 + c < C) ? *reinterpret_cast<const float4 *>(cent + (int64_t)(c0 + c) * dn + k0 + k4)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    };
-    auto store = [&]() {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int idx = tid + q * 256, c = idx & (kTC - 1), k4 = (idx >> 7) * 4;
-            cs[(k4 + 0) * kTC + c] = pre[q].x;
-            cs[(k4 + 1) * kTC + c] = pre[q].y;
-            cs[(k4 + 2) * kTC + c] = pre[q].z;
-            cs[(k4 + 3) * kTC + c] = pre[q].w;
-        }
-    };
-    fetch(0, 0);
-    for (int c0 = 0; c0 < C; c0 += kTC) {
-        float acc[8][8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-        for (int ks = 0; ks < nslices; ++ks) {
-            __syncthreads();  // previous slice consumed
-            store();
-            __syncthreads();
-            // prefetch the next slice (this chunk, or the next chunk's first)
-            if (ks + 1 < nslices) fetch(c0, (ks + 1) * kKS);
-            else if (c0 + kTC < C) fetch(c0 + kTC, 0);
-            const float *xk = xs + ks * kKS * kTP + ty * 8;
-#pragma unroll 4
-            for (int k = 0; k < kKS; ++k) {
-                const float4 x0 = *reinterpret_cast<const float4 *>(xk + k * kTP);
-                const float4 x1 = *reinterpret_cast<const float4 *>(xk + k * kTP + 4);
-                const float4 w0 = *reinterpret_cast<const float4 *>(cs + k * kTC + tx * 4);
-                const float4 w1 = *reinterpret_cast<const float4 *>(cs + k * kTC + 64 + tx * 4);
-                const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                const float cv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xv[i], cv[j], acc[i][j]);
-            }
-        }
-        // scores of this chunk -> per-row (best, arg, second) over the 16 lanes
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float b1 = INFINITY, b2 = INFINITY;
-            int a1 = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int c = c0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
-                if (c < C) better(b1, a1, b2, fmaf(-2.f, acc[i][j], cn[c]), c);
-            }
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) {
-                const float ob1 = __shfl_xor_sync(0xffffffffu, b1, o);
-                const float ob2 = __shfl_xor_sync(0xffffffffu, b2, o);
-                const int oa1 = __shfl_xor_sync(0xffffffffu, a1, o);
-                better(b1, a1, b2, ob1, oa1);
-                b2 = fminf(b2, ob2);
-            }
-            if (tx == i) {
-                better(rb1, ra1, rb2, b1, a1);
-                rb2 = fminf(rb2, b2);
-            }
-        }
-    }
-    const int n = p0 + ty * 8 + tx;
-    if (tx < 8 && n < N) {
-        const float xn = sqrtf(xnorm2[(int64_t)bh * N + n]);
-        const float R = sqrtf(r2);
-        const float B = (float)(dn + 2) * 5.9604645e-8f * (2.f * xn * R + r2) * 1.01f + 1e-30f;
-        P.labels[(int64_t)bh * N + n] = ra1;
-        if (!(rb2 - rb1 > 2.f * B)) {
-            const int slot = atomicAdd(fix_count, 1);
-            fix_list[slot] = bh * N + n;
-        }
-    }
-}
-
+// -------------------------------------------------------------- assign fix-up
+// The tensor-core query assignment (kmeans_tc.cu) lists the rows whose best
+// and second-best expanded-form scores lie within its fp32 error margin.
 // Exact re-decision of the listed rows: fp64 direct-form distance to every
 // centroid, lowest index on ties.  One warp per row.
 __global__ void __launch_bounds__(256) km_fixup_kernel(KmProblem P, int N, int D, const int32_t *fix_list,
@@ -632,9 +473,7 @@ cudaError_t km_configure()
 {
     cudaError_t e = cudaFuncSetAttribute(km_assign_direct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)direct_smem(128));
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(km_assign_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (128 * kTP + kKS * kTC) * (int)sizeof(float));
+    return e;
 }
 
 void launch_km_init(const KmBatch &b, int BH, int N, int D, uint32_t seed, cudaStream_t st)
@@ -647,17 +486,6 @@ void launch_km_assign_direct(const KmBatch &b, int BH, int N, int D, cudaStream_
 {
     km_assign_direct_kernel<<<dim3((N + kDirRows - 1) / kDirRows, BH, b.count), kDirRows / 2,
                               direct_smem(max_dim(b)), st>>>(b, N, D);
-    count_launches(1);
-}
-
-void launch_km_assign_tiled(const KmProblem &P, int BH, int N, int D, const float *xnorm2, int32_t *fix_list,
-                            int32_t *fix_count, cudaStream_t st)
-{
-    cudaMemsetAsync(fix_count, 0, sizeof(int32_t), st);
-    km_assign_tiled_kernel<<<dim3((N + kTP - 1) / kTP, BH), 256, (size_t)(P.dim_n * kTP + kKS * kTC) * sizeof(float), st>>>(
-        P, N, D, xnorm2, fix_list, fix_count);
-    count_launches(1);
-    km_fixup_kernel<<<148 * 4, 256, 0, st>>>(P, N, D, fix_list, fix_count);
     count_launches(1);
 }
 

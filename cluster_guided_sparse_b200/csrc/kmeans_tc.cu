@@ -1,5 +1,6 @@
-// Query k-means assignment on the 5th-generation tensor cores, with the same
-// certified result as the fp32 register-tiled kernel.
+// Query k-means assignment on the 5th-generation tensor cores.  The labels
+// are certified: they equal the argmin of exact arithmetic on the stored fp32
+// centroids and bf16 rows (lowest index on ties).
 //
 // The assignment score e_j = ||c_j||^2 - 2 x.c_j needs x.c_j for every row
 // and centroid: a dense contraction (N x d times d x C per head).  The rows x

@@ -24,7 +24,6 @@ void launch_km_assign_direct(const KmBatch &, int, int, int, cudaStream_t);
 void launch_km_sort(const KmBatch &, int, int, cudaStream_t);
 void launch_bisect(const __nv_bfloat16 *, int, int, int, int, int, int32_t *, int32_t *, double *, int32_t *, float *,
                    float *, int32_t *, int32_t *, int32_t *, cudaStream_t);
-void launch_km_assign_tiled(const KmProblem &, int, int, int, const float *, int32_t *, int32_t *, cudaStream_t);
 cudaError_t km_tc_configure();
 bool launch_km_assign_tc(const KmProblem &, __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, const float *, int32_t *,
                          int32_t *, int32_t *, cudaStream_t);
@@ -411,7 +410,7 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     // as one batch on the direct-form kernel; queries with >= 128 clusters use
     // the certified tensor-core kernel (bf16 hi/lo centroid split, fp64 fix-up
     // of the rows inside its error margin).
-    const bool tiled_q = L.Cq >= 128;
+    const bool tc_q = L.Cq >= 128;
     KmBatch all{};
     for (int i = 0; i < 3; ++i) all.p[i] = key_problem(L, ws, i);
     all.p[3] = query_problem(L, ws);
@@ -425,7 +424,7 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     int32_t *fix_list = fix_count + 4;
     bool tc_ok = true;
     auto assign = [&]() {
-        if (tiled_q) {
+        if (tc_q) {
             launch_km_assign_direct(keys, BH, N, D, s);
             tc_ok = tc_ok && launch_km_assign_tc(all.p[3], at<__nv_bfloat16>(ws, L.q_chi), at<__nv_bfloat16>(ws, L.q_clo),
                                                  BH, N, D, at<float>(ws, L.qnorm), fix_list, fix_count,
