@@ -144,12 +144,33 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (a device tensor under NCCL, a
+    host tensor under gloo)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_ms_per_call(rank_ms: float, steps: int, world: int) -> float:
+    """Whole-job ms per call: every rank made `steps` calls inside its timed
+    region; the job's time is the slowest rank's."""
+    return max_over_ranks(rank_ms, world) / (steps * world)
+
+
+def tile_flops(sizes: torch.Tensor, n: torch.Tensor, d: int, bm: int = 128, bn: int = 128,
+               item_rows: int = 256) -> float:
+    """Flops of the tiles the attention kernel issues: each cluster's queries
+    in work items of up to `item_rows`, each item's rows padded to `bm`-row Q
+    tiles, its key list padded to `bn`-key tiles (Q.K^T plus P.V)."""
+    s = sizes.to(torch.int64)
+    full, rem = s // item_rows, s % item_rows
+    qtiles = full * (item_rows // bm) + (rem + bm - 1) // bm
+    ktiles = (n.to(torch.int64) + bn - 1) // bn
+    return 4.0 * d * bm * bn * float((qtiles * ktiles).sum())
 
 
 # --------------------------------------------------------------------------- oracle sample
@@ -283,10 +304,11 @@ def run_scope(args, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
     launches = scope.lib().scope_kernel_launches() - L0
-    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    ms_per_call = job_ms_per_call(t0.elapsed_time(t1), args.steps, world)
+    total_ms = ms_per_call * args.steps * world
     plan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    ms_per_call = total_ms / (args.steps * world)
+    call_median_ms = statistics.median(e[0].elapsed_time(e[2]) for e in ev)
 
     # algorithmic attention flops of one launch: 4 d sum_c |c| n_c
     sizes = pl.view("q_sizes").to(torch.int64)
@@ -296,6 +318,7 @@ def run_scope(args, world, rank, local):
     density = pairs / (w.B * w.H * float(w.N) ** 2)
     hbm, bf16, bf16_sus, src = peaks()
     achieved = attn_flops / (attn_ms * 1e-3) / 1e12
+    tile_tf = tile_flops(sizes.flatten(), n.flatten(), w.D) / (attn_ms * 1e-3) / 1e12
 
     # this build's dense attention (RoPE + all keys) at the same shape, for context
     od = torch.empty_like(o)
@@ -346,7 +369,8 @@ def run_scope(args, world, rank, local):
         "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N, "heads": w.H,
                    "head_dim": w.D, "top_p": w.top_p, "online_topk": bool(w.online_topk),
                    "l2": "inputs 2.2 GB >> 126 MB L2, no flush", "parallelism": f"replicas x{world}"},
-        "effective_tflops": eff, "plan_ms": plan_ms, "attn_ms": attn_ms, "density": density,
+        "effective_tflops": eff, "plan_ms": plan_ms, "attn_ms": attn_ms, "call_median_ms": call_median_ms,
+        "density": density, "tile_tflops": tile_tf, "tile_frac_of_sustained": tile_tf / bf16_sus,
         "own_dense_ms": dense_ms, "speedup_vs_own_dense": dense_ms / ms_per_call,
         "roofline": {"kernel": "sparse attention (scope_attn)", "bound": "tensor", "achieved": achieved,
                      "peak": bf16_sus, "unit": "TFLOP/s", "frac": achieved / bf16_sus,
