@@ -26,10 +26,11 @@
 // when a row's max grows by more than 2^8, so P never exceeds 256.
 //
 // The softmax loads its 128-wide S row with four back-to-back tcgen05.ld
-// (one wait) for the row max, reloads it in two halves for the exponentials,
-// and does the scale/subtract and the row sum with packed f32x2 instructions.
-// (Moving a third of the exponentials to a cubic on the FMA pipe was slower
-// here: the softmax is latency-bound, not MUFU-bound.)
+// (one wait) and keeps it in registers: a three-input max for the row max,
+// then the scale/subtract and the row sum as packed f32x2 instructions on
+// 64-bit registers.  (Moving a third of the exponentials to a cubic on the
+// FMA pipe, and handing P to the issuer in two 64-key halves, were both
+// slower here.)
 //
 // Every mbarrier wait is bounded (about two seconds of clock64); on timeout
 // the thread records SCOPE's timeout bit in the device error word, the CTA
