@@ -32,15 +32,16 @@ void launch_km_reduce(const KmBatch &, int, int, int, cudaStream_t);
 struct SelArgs;
 void launch_lut(const float *, const float *, const float *, const float *, float *, int, int, int, int, int, int,
                 int, int, int, cudaStream_t);
-void launch_items(const int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, int, int, int, int, int, int,
-                  cudaStream_t);
+void launch_items(const int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, uint16_t *, int, int, int, int, int,
+                  int, cudaStream_t);
+cudaError_t select_configure();
 cudaError_t attn_tc_configure();
 int attn_tc_max_items(int BH, int N, int Cq);
 bool launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, __nv_bfloat16 *, int4 *,
                     int32_t *, int, const int32_t *, const int32_t *, const int32_t *, const long long *,
                     const int32_t *, const int32_t *, int32_t *, int, int, int, int, cudaStream_t);
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
-                   const int32_t *item_n, int Pcap, int N, int Cq, int Ct, int Ch, int Cw, int BH, float top_p,
+                   const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch, int Cw, int BH, float top_p,
                    float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes, int32_t *r, int32_t *n,
                    int32_t *kh, long long *offsets, int32_t *indices, int online, cudaStream_t st);
 }  // namespace scope
@@ -80,7 +81,7 @@ struct Layout {
     int64_t cap;
     size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
-    size_t lut, item_hist, item_id, item_cnt, item_n, r, n, kh, offsets, indices, work, nwork, vb, fix;
+    size_t lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
     size_t bis_order, bis_delta, q_chi, q_clo, q_sums, k_sums[3], sums_bytes;
     size_t total;
 };
@@ -251,6 +252,7 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.item_id = take(cur, BH * L.Pcap * 4);
     L.item_cnt = take(cur, BH * L.Pcap * 4);
     L.item_n = take(cur, BH * 4);
+    L.key_item = take(cur, BH * N * 2);
     L.r = take(cur, BH * L.Cq * 4);
     L.n = take(cur, BH * L.Cq * 4);
     L.kh = take(cur, BH * 4);
@@ -272,7 +274,8 @@ scope_status check_device(cudaStream_t)
     if (major != 10) return fail(SCOPE_EDEVICE, "libscope.so is built for sm_100a; device has compute capability %d.x", major);
     static bool configured[64] = {false};
     if (dev < 64 && !configured[dev]) {
-        if (km_configure() != cudaSuccess || attn_tc_configure() != cudaSuccess || km_tc_configure() != cudaSuccess)
+        if (km_configure() != cudaSuccess || attn_tc_configure() != cudaSuccess || km_tc_configure() != cudaSuccess ||
+            select_configure() != cudaSuccess)
             return fail(SCOPE_ECUDA, "kernel attribute setup failed");
         configured[dev] = true;
     }
@@ -450,10 +453,11 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
                at<float>(ws, L.k_cent[2]), at<float>(ws, L.lut), BH, L.Cq, D, L.ds[0], L.ds[1], L.ds[2], L.C[0],
                L.C[1], L.C[2], s);
     launch_items(at<int32_t>(ws, L.k_codes), at<int32_t>(ws, L.item_hist), at<int32_t>(ws, L.item_id),
-                 at<int32_t>(ws, L.item_cnt), at<int32_t>(ws, L.item_n), BH, N, L.C[1], L.C[2], L.P, L.Pcap, s);
+                 at<int32_t>(ws, L.item_cnt), at<int32_t>(ws, L.item_n), at<uint16_t>(ws, L.key_item), BH, N, L.C[1],
+                 L.C[2], L.P, L.Pcap, s);
     run_selection(at<float>(ws, L.lut), at<int32_t>(ws, L.k_codes), at<int32_t>(ws, L.item_id),
-                  at<int32_t>(ws, L.item_cnt), at<int32_t>(ws, L.item_n), L.Pcap, N, L.Cq, L.C[0], L.C[1], L.C[2],
-                  BH, p->top_p, 1.0f / sqrtf((float)D), p->k_min, at<int32_t>(ws, L.stats) + 4,
+                  at<int32_t>(ws, L.item_cnt), at<int32_t>(ws, L.item_n), at<uint16_t>(ws, L.key_item), L.Pcap, N,
+                  L.Cq, L.C[0], L.C[1], L.C[2], BH, p->top_p, 1.0f / sqrtf((float)D), p->k_min, at<int32_t>(ws, L.stats) + 4,
                   at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.r), at<int32_t>(ws, L.n), at<int32_t>(ws, L.kh),
                   at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, s);
     if ((st = launch_status("selection")) != SCOPE_OK) return st;

@@ -29,6 +29,7 @@ struct SelArgs {
     const int32_t *item_id;   // [BH][Pcap] distinct code triples, ascending
     const int32_t *item_cnt;  // [BH][Pcap]
     const int32_t *item_n;    // [BH]
+    const uint16_t *key_item; // [BH][N] rank of each key's triple among the head's items
     int Pcap, N, Cq, Ct, Ch, Cw, BH;
     float top_p, inv_sqrt_d;
     int k_min;
@@ -75,13 +76,14 @@ __global__ void item_hist_kernel(const int32_t *codes, int32_t *hist, int N, int
     atomicAdd(&hist[(int64_t)bh * P + id], 1);
 }
 
-// Ordered compaction of the non-empty triples of one head.
-__global__ void __launch_bounds__(1024) item_compact_kernel(const int32_t *hist, int32_t *item_id,
-                                                            int32_t *item_cnt, int32_t *item_n, int P, int Pcap)
+// Ordered compaction of the non-empty triples of one head; the histogram
+// entry of each non-empty triple is replaced by its item rank.
+__global__ void __launch_bounds__(1024) item_compact_kernel(int32_t *hist, int32_t *item_id, int32_t *item_cnt,
+                                                            int32_t *item_n, int P, int Pcap)
 {
     __shared__ int tmp[33];
     const int bh = blockIdx.x;
-    const int32_t *h = hist + (int64_t)bh * P;
+    int32_t *h = hist + (int64_t)bh * P;
     int carry = 0;
     for (int base = 0; base < P; base += blockDim.x) {
         const int i = base + threadIdx.x;
@@ -91,10 +93,24 @@ __global__ void __launch_bounds__(1024) item_compact_kernel(const int32_t *hist,
         if (cnt > 0) {
             item_id[(int64_t)bh * Pcap + carry + ex] = i;
             item_cnt[(int64_t)bh * Pcap + carry + ex] = cnt;
+            h[i] = carry + ex;
         }
         carry += tot;
     }
     if (threadIdx.x == 0) item_n[bh] = carry;
+}
+
+// Item rank of every key (P <= 65536, so a rank fits 16 bits).
+__global__ void key_item_kernel(const int32_t *codes, const int32_t *rank, uint16_t *key_item, int N, int BH, int Ch,
+                                int Cw, int P)
+{
+    const int bh = blockIdx.y;
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    const int64_t plane = (int64_t)BH * N;
+    const int64_t i = (int64_t)bh * N + n;
+    const int id = (codes[i] * Ch + codes[plane + i]) * Cw + codes[2 * plane + i];
+    key_item[i] = (uint16_t)rank[(int64_t)bh * P + id];
 }
 
 // -------------------------------------------------------------- radix select
@@ -311,10 +327,14 @@ __global__ void __launch_bounds__(1024) topk_kernel(const int32_t *sizes, const 
 // above the cut score, then the lowest-index `need` keys at the cut score.
 // Written in ascending key order: the output slot of key j is
 // (#keys above the cut before j) + min(#keys at the cut before j, need).
+// A key's side of the cut is its item's, so the items are classed once in
+// shared memory (2 above, 1 at, 0 below) and each key costs one 16-bit load.
+constexpr int kEmitPer = 8;
+
 __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int32_t *n_in,
                                                            const long long *offsets, int32_t *indices)
 {
-    extern __shared__ float L[];
+    extern __shared__ __align__(16) float L[];
     __shared__ SelShared S;
     __shared__ unsigned ptmp[33];
     const int c = blockIdx.x, bh = blockIdx.y;
@@ -327,6 +347,7 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         return;
     }
     const int Csum = a.Ct + a.Ch + a.Cw;
+    uint8_t *cls = reinterpret_cast<uint8_t *>(L + ((Csum + 3) & ~3));
     const float *lrow = a.lut + bhc * Csum;
     for (int e = threadIdx.x; e < Csum; e += blockDim.x) L[e] = lrow[e];
     __syncthreads();
@@ -339,42 +360,44 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         if (threadIdx.x == 0) set_error(a.err, kErrRange, 0x200 + c);
         return;
     }
-    const int64_t plane = (int64_t)a.BH * a.N;
-    const int32_t *ct = a.codes + (int64_t)bh * a.N;
-    const int32_t *ch = ct + plane;
-    const int32_t *cw = ct + 2 * plane;
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const uint32_t u = ordered_key(item_score(L, ids[i], a.Ch, a.Cw, a.Ct));
+        cls[i] = u > cut ? 2 : (u == cut ? 1 : 0);
+    }
+    __syncthreads();
+    const uint16_t *ki = a.key_item + (int64_t)bh * a.N;
+    const bool vec = (((int64_t)bh * a.N) & 7) == 0;  // 16-byte aligned rows of 8 ranks
     int gt_run = 0, eq_run = 0;
-    constexpr int PER = 4;
-    for (int base = 0; base < a.N; base += kSelThreads * PER) {
-        const int j0 = base + threadIdx.x * PER;
+    for (int base = 0; base < a.N; base += kSelThreads * kEmitPer) {
+        const int j0 = base + threadIdx.x * kEmitPer;
         unsigned gt = 0, eq = 0;
-        uint32_t u[PER];
+        uint8_t k[kEmitPer];
+        if (vec && j0 + kEmitPer <= a.N) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(ki + j0);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int t = 0; t < PER; ++t) {
-            const int j = j0 + t;
-            u[t] = 0u;
-            if (j < a.N) {
-                const float s = (L[ct[j]] + L[a.Ct + ch[j]]) + L[a.Ct + a.Ch + cw[j]];
-                u[t] = ordered_key(s);
-                gt += u[t] > cut;
-                eq += u[t] == cut;
-            } else {
-                u[t] = 0u;
-            }
+            for (int t = 0; t < kEmitPer; ++t) k[t] = cls[(ws[t >> 1] >> (16 * (t & 1))) & 0xffffu];
+        } else {
+#pragma unroll
+            for (int t = 0; t < kEmitPer; ++t) k[t] = j0 + t < a.N ? cls[ki[j0 + t]] : 0;
+        }
+#pragma unroll
+        for (int t = 0; t < kEmitPer; ++t) {
+            gt += k[t] == 2;
+            eq += k[t] == 1;
         }
         unsigned tot;
         const unsigned ex = block_excl_scan(gt | (eq << 16), ptmp, tot);
         unsigned g = gt_run + (ex & 0xffffu), e = eq_run + (ex >> 16);
 #pragma unroll
-        for (int t = 0; t < PER; ++t) {
+        for (int t = 0; t < kEmitPer; ++t) {
             const int j = j0 + t;
-            if (j >= a.N) break;
-            if (u[t] > cut) {
+            if (k[t] == 2) {
                 const unsigned slot = g + (e < (unsigned)need ? e : (unsigned)need);
                 if (slot < (unsigned)n) out[slot] = j;
                 else set_error(a.err, kErrRange, 0x300 + c);
                 ++g;
-            } else if (u[t] == cut) {
+            } else if (k[t] == 1) {
                 if (e < (unsigned)need) {
                     if (g + e < (unsigned)n) out[g + e] = j;
                     else set_error(a.err, kErrRange, 0x300 + c);
@@ -387,6 +410,14 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
     }
 }
 
+static size_t emit_smem(int Csum, int Pcap) { return (size_t)((Csum + 3) & ~3) * sizeof(float) + (size_t)Pcap; }
+
+cudaError_t select_configure()
+{
+    return cudaFuncSetAttribute(emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)emit_smem(3 * kMaxClusters, kMaxItems));
+}
+
 // -------------------------------------------------------------- launchers
 void launch_lut(const float *qcent, const float *kc_t, const float *kc_h, const float *kc_w, float *lut, int BH,
                 int Cq, int D, int dt, int dh, int dw, int Ct, int Ch, int Cw, cudaStream_t st)
@@ -397,12 +428,14 @@ void launch_lut(const float *qcent, const float *kc_t, const float *kc_h, const 
 }
 
 void launch_items(const int32_t *codes, int32_t *hist, int32_t *item_id, int32_t *item_cnt, int32_t *item_n,
-                  int BH, int N, int Ch, int Cw, int P, int Pcap, cudaStream_t st)
+                  uint16_t *key_item, int BH, int N, int Ch, int Cw, int P, int Pcap, cudaStream_t st)
 {
     cudaMemsetAsync(hist, 0, (size_t)BH * P * sizeof(int32_t), st);
     item_hist_kernel<<<dim3((N + 255) / 256, BH), 256, 0, st>>>(codes, hist, N, BH, Ch, Cw, P);
     count_launches(1);
     item_compact_kernel<<<BH, 1024, 0, st>>>(hist, item_id, item_cnt, item_n, P, Pcap);
+    count_launches(1);
+    key_item_kernel<<<dim3((N + 255) / 256, BH), 256, 0, st>>>(codes, hist, key_item, N, BH, Ch, Cw, P);
     count_launches(1);
 }
 
@@ -422,13 +455,13 @@ void launch_topk(const int32_t *sizes, const int32_t *r, int32_t *n_out, int32_t
 
 void launch_emit(const SelArgs &a, const int32_t *n_in, const long long *offsets, int32_t *indices, cudaStream_t st)
 {
-    const size_t smem = (size_t)(a.Ct + a.Ch + a.Cw) * sizeof(float);
+    const size_t smem = emit_smem(a.Ct + a.Ch + a.Cw, a.Pcap);
     emit_kernel<<<dim3(a.Cq, a.BH), kSelThreads, smem, st>>>(a, n_in, offsets, indices);
     count_launches(1);
 }
 
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
-                   const int32_t *item_n, int Pcap, int N, int Cq, int Ct, int Ch, int Cw, int BH, float top_p,
+                   const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch, int Cw, int BH, float top_p,
                    float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes, int32_t *r, int32_t *n,
                    int32_t *kh, long long *offsets, int32_t *indices, int online, cudaStream_t st)
 {
@@ -438,6 +471,7 @@ void run_selection(const float *lut, const int32_t *codes, const int32_t *item_i
     a.item_id = item_id;
     a.item_cnt = item_cnt;
     a.item_n = item_n;
+    a.key_item = key_item;
     a.Pcap = Pcap;
     a.N = N;
     a.Cq = Cq;
