@@ -74,6 +74,7 @@ def lib():
         L.orc_emit.argtypes = [_d, _I, _I, _i32]
         L.orc_attn_rows.argtypes = [_d, _I, _d, _d, _I, _i32, _I, ctypes.c_double, _d]
         L.orc_bisect.argtypes = [_d, _I, _I, _I, ctypes.c_int, _i32, _d, _i64]
+        L.orc_attn_rows_comp.argtypes = [_d, _I, _d, _d, _I, _I, _i32, _I, _i32, _I, ctypes.c_double, _d]
         L.orc_bisect.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -204,6 +205,20 @@ def attention_rows(q_rows, K, V, sel, scale: float) -> np.ndarray:
     sel = np.ascontiguousarray(sel, np.int32)
     o = np.empty_like(q_rows)
     lib().orc_attn_rows(q_rows, q_rows.shape[0], K, V, K.shape[1], sel, sel.shape[0], float(scale), o)
+    return o
+
+
+def attention_rows_comp(q_rows, K, V, sel, klab, scale: float) -> np.ndarray:
+    """Attention over the selected keys plus every excluded key entering through
+    its key cluster's mean key and mean value (ClusterAttention compensation,
+    reading R16); klab[j] is key j's cluster."""
+    q_rows, K, V = _f64(q_rows), _f64(K), _f64(V)
+    sel = np.ascontiguousarray(sel, np.int32)
+    klab = np.ascontiguousarray(klab, np.int32)
+    C = int(klab.max()) + 1 if klab.size else 0
+    o = np.empty_like(q_rows)
+    lib().orc_attn_rows_comp(q_rows, q_rows.shape[0], K, V, K.shape[0], K.shape[1], sel, sel.shape[0], klab, C,
+                             float(scale), o)
     return o
 
 

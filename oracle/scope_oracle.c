@@ -12,7 +12,7 @@
  *   [CLUSTER] "ClusterAttention: A training-free speedup of bidirectional
  *             attention", abstract.
  * The pages are abstract-level; every concrete choice below that they leave
- * open is a stated reading (R1..R14) listed beside the function it affects.
+ * open is a stated reading (R1..R16) listed beside the function it affects.
  *
  * Conventions: one (batch, head) at a time; row-major [rows][D] arrays of
  * double; labels int32; counts int64.  Every function is single-threaded and
@@ -324,6 +324,83 @@ void orc_attn_rows(const double *q, int64_t nq, const double *K, const double *V
         }
     }
     free(lg);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Compensation of excluded clusters [CLUSTER: "compensation of excluded     */
+/* clusters through their mean"].                                            */
+/* R16: key cluster k (klab) has mean key mu_k and mean value vbar_k over    */
+/*      all of its members.  For one query cluster with selected keys S, m_k */
+/*      is the number of members of k not in S; every such key enters the   */
+/*      softmax through its cluster's mean:                                  */
+/*        o = (sum_{j in S} e^{a_j} v_j + sum_k m_k e^{b_k} vbar_k)          */
+/*          / (sum_{j in S} e^{a_j} + sum_k m_k e^{b_k}),                    */
+/*      a_j = scale q.k_j, b_k = scale q.mu_k.  With every cluster a single  */
+/*      key, or with identical keys and values inside each cluster, this is  */
+/*      dense attention.                                                    */
+/* ------------------------------------------------------------------------ */
+void orc_attn_rows_comp(const double *q, int64_t nq, const double *K, const double *V, int64_t N, int64_t D,
+                        const int32_t *sel, int64_t n, const int32_t *klab, int64_t C, double scale, double *o)
+{
+    double *mu = (double *)calloc((size_t)(C * D), sizeof(double));
+    double *vb = (double *)calloc((size_t)(C * D), sizeof(double));
+    int64_t *size = (int64_t *)calloc((size_t)C, sizeof(int64_t));
+    int64_t *m = (int64_t *)calloc((size_t)C, sizeof(int64_t));
+    for (int64_t j = 0; j < N; ++j) {
+        const int64_t k = klab[j];
+        size[k] += 1;
+        for (int64_t d = 0; d < D; ++d) {
+            mu[k * D + d] += K[j * D + d];
+            vb[k * D + d] += V[j * D + d];
+        }
+    }
+    for (int64_t k = 0; k < C; ++k)
+        for (int64_t d = 0; d < D; ++d) {
+            if (size[k] > 0) {
+                mu[k * D + d] /= (double)size[k];
+                vb[k * D + d] /= (double)size[k];
+            }
+        }
+    for (int64_t k = 0; k < C; ++k) m[k] = size[k];
+    for (int64_t t = 0; t < n; ++t) m[klab[sel[t]]] -= 1;
+    double *lg = (double *)malloc((size_t)(n + C > 0 ? n + C : 1) * sizeof(double));
+    for (int64_t i = 0; i < nq; ++i) {
+        const double *qi = q + i * D;
+        double mx = -INFINITY;
+        for (int64_t t = 0; t < n; ++t) {
+            double dot = 0.0;
+            for (int64_t d = 0; d < D; ++d) dot += qi[d] * K[(int64_t)sel[t] * D + d];
+            lg[t] = dot * scale;
+            if (lg[t] > mx) mx = lg[t];
+        }
+        for (int64_t k = 0; k < C; ++k) {
+            if (m[k] <= 0) continue;
+            double dot = 0.0;
+            for (int64_t d = 0; d < D; ++d) dot += qi[d] * mu[k * D + d];
+            lg[n + k] = dot * scale;
+            if (lg[n + k] > mx) mx = lg[n + k];
+        }
+        double den = 0.0;
+        double *oi = o + i * D;
+        for (int64_t d = 0; d < D; ++d) oi[d] = 0.0;
+        for (int64_t t = 0; t < n; ++t) {
+            const double w = exp(lg[t] - mx);
+            den += w;
+            for (int64_t d = 0; d < D; ++d) oi[d] += w * V[(int64_t)sel[t] * D + d];
+        }
+        for (int64_t k = 0; k < C; ++k) {
+            if (m[k] <= 0) continue;
+            const double w = (double)m[k] * exp(lg[n + k] - mx);
+            den += w;
+            for (int64_t d = 0; d < D; ++d) oi[d] += w * vb[k * D + d];
+        }
+        for (int64_t d = 0; d < D; ++d) oi[d] /= den;
+    }
+    free(lg);
+    free(m);
+    free(size);
+    free(vb);
+    free(mu);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -272,6 +272,48 @@ def test_bisect_median_split_ties_by_token():
     assert lab.tolist() == [0, 0, 1, 1, 2, 2, 3, 3]
 
 
+# ----------------------------------------------------------------------------- compensation
+# ClusterAttention, abstract: excluded clusters are compensated through their
+# mean.  Where a cluster's members are indistinguishable from its mean, the
+# compensated attention must equal dense attention whatever is selected.
+def test_compensation_with_single_key_clusters_is_dense():
+    rng = np.random.default_rng(11)
+    N, D = 48, 8
+    K, V, q = rng.standard_normal((N, D)), rng.standard_normal((N, D)), rng.standard_normal((5, D))
+    dense = oracle.dense_attention(q, K, V)
+    for sel in (np.array([], np.int32), np.array([3], np.int32), np.sort(rng.choice(N, 17, replace=False))):
+        o = oracle.attention_rows_comp(q, K, V, sel.astype(np.int32), np.arange(N), 1 / np.sqrt(D))
+        np.testing.assert_allclose(o, dense, rtol=1e-12, atol=1e-12)
+
+
+def test_compensation_with_identical_members_is_dense():
+    # 6 clusters of 4 identical keys (and identical values): an excluded
+    # member counts exactly like the key it copies, so m_k must weight it.
+    rng = np.random.default_rng(12)
+    C, M, D = 6, 4, 5
+    Kc, Vc = 2 * rng.standard_normal((C, D)), rng.standard_normal((C, D))
+    klab = np.repeat(np.arange(C), M).astype(np.int32)
+    K, V = Kc[klab], Vc[klab]
+    q = rng.standard_normal((3, D))
+    dense = oracle.dense_attention(q, K, V)
+    # select all of cluster 0, one member of cluster 2, nothing else
+    sel = np.array([0, 1, 2, 3, 9], np.int32)
+    o = oracle.attention_rows_comp(q, K, V, sel, klab, 1 / np.sqrt(D))
+    np.testing.assert_allclose(o, dense, rtol=1e-12, atol=1e-12)
+    # the uncompensated sparse result differs (the excluded keys carry mass)
+    assert np.abs(oracle.attention_rows(q, K, V, sel, 1 / np.sqrt(D)) - dense).max() > 1e-3
+
+
+def test_compensation_with_everything_selected_is_plain_attention():
+    rng = np.random.default_rng(13)
+    N, D = 32, 6
+    K, V, q = rng.standard_normal((N, D)), rng.standard_normal((N, D)), rng.standard_normal((4, D))
+    klab = (np.arange(N) // 8).astype(np.int32)
+    sel = np.arange(N, dtype=np.int32)
+    np.testing.assert_allclose(oracle.attention_rows_comp(q, K, V, sel, klab, 0.4),
+                               oracle.attention_rows(q, K, V, sel, 0.4), rtol=1e-12, atol=1e-12)
+
+
 # ----------------------------------------------------------------------------- pipeline
 def test_pipeline_tiny_config_invariants():
     w = synth.WORKLOADS["tiny"]
