@@ -44,7 +44,8 @@ class ScopeParams(ctypes.Structure):
                 ("theta", ctypes.c_double), ("c_q", ctypes.c_int32), ("c_t", ctypes.c_int32),
                 ("c_h", ctypes.c_int32), ("c_w", ctypes.c_int32), ("iters", ctypes.c_int32),
                 ("init_seed", ctypes.c_uint32), ("top_p", ctypes.c_float), ("k_min", ctypes.c_int32),
-                ("online_topk", ctypes.c_int32), ("fixed_cluster_size", ctypes.c_int32)]
+                ("online_topk", ctypes.c_int32), ("fixed_cluster_size", ctypes.c_int32),
+                ("compensate", ctypes.c_int32)]
 
 
 class ScopeView(ctypes.Structure):
@@ -129,7 +130,8 @@ def make_params(w=None, **kw):
     if w is not None:
         f = dict(d_t=w.d_split[0], d_h=w.d_split[1], d_w=w.d_split[2], theta=w.theta, c_q=w.c_q,
                  c_t=w.c_sub[0], c_h=w.c_sub[1], c_w=w.c_sub[2], iters=w.iters, init_seed=0, top_p=w.top_p,
-                 k_min=w.k_min, online_topk=w.online_topk, fixed_cluster_size=w.fixed_cluster_size)
+                 k_min=w.k_min, online_topk=w.online_topk, fixed_cluster_size=w.fixed_cluster_size,
+                 compensate=w.compensate)
         grid = tuple(w.grid)
     else:
         grid = (0, 0, 0)

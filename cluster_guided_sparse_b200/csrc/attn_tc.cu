@@ -65,6 +65,7 @@ struct Args {
     const int32_t *indices;
     const int32_t *n_c;        // [BH][Cq] or null
     int32_t *err;
+    float *lse;                // [BH][N] natural log-sum-exp of every stored row, or null
     int N, Cq;
     float scale_log2;          // log2(e) / sqrt(D)
 };
@@ -348,6 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool store = qi < nq;
             const int tok = store ? (a.perm ? a.perm[base + cstart + q0 + qi] : q0 + qi) : 0;
             const float inv = 1.f / l;
+            // row log-sum-exp, natural log: the row's exponentials are 2^(s*scale*log2e - m_run)
+            if (a.lse && store) a.lse[base + tok] = (m_run + log2f(l)) * 0.6931471805599453f;
             __nv_bfloat16 *dst = a.o + (base + tok) * D;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
@@ -441,7 +444,7 @@ bool rows_tensor_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int
 bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv_bfloat16 *v, __nv_bfloat16 *o,
                     int4 *items, int32_t *n_items, int max_items, const int32_t *sizes, const int32_t *perm,
                     const int32_t *start, const long long *offsets, const int32_t *indices, const int32_t *n_c,
-                    int32_t *err, int BH, int N, int D, int Cq, cudaStream_t st)
+                    int32_t *err, float *lse, int BH, int N, int D, int Cq, cudaStream_t st)
 {
     CUtensorMap tmK, tmV;
     if (!rows_tensor_map(&tmK, kr, (uint64_t)BH * N, D, 1) || !rows_tensor_map(&tmV, v, (uint64_t)BH * N, D, 1))
@@ -461,6 +464,7 @@ bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv
     a.indices = indices;
     a.n_c = n_c;
     a.err = err;
+    a.lse = lse;
     a.N = N;
     a.Cq = Cq;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)D);

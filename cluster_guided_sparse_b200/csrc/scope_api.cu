@@ -39,9 +39,14 @@ cudaError_t attn_tc_configure();
 int attn_tc_max_items(int BH, int N, int Cq);
 bool launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, __nv_bfloat16 *, int4 *,
                     int32_t *, int, const int32_t *, const int32_t *, const int32_t *, const long long *,
-                    const int32_t *, const int32_t *, int32_t *, int, int, int, int, cudaStream_t);
+                    const int32_t *, const int32_t *, int32_t *, float *, int, int, int, int, cudaStream_t);
+void launch_compensate(const __nv_bfloat16 *, const __nv_bfloat16 *, const int32_t *, const int32_t *, const int32_t *,
+                       const int32_t *, const int32_t *, const int32_t *, const float *, float *, const long long *,
+                       const int32_t *, const int32_t *, const float *, __nv_bfloat16 *, int, int, int, int, int,
+                       cudaStream_t);
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
-                   const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch, int Cw, int BH, float top_p,
+                   const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch, int Cw,
+                   int BH, float top_p,
                    float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes, int32_t *r, int32_t *n,
                    int32_t *kh, long long *offsets, int32_t *indices, int online, cudaStream_t st);
 }  // namespace scope
@@ -82,7 +87,8 @@ struct Layout {
     size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
     size_t lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
-    size_t bis_order, bis_delta, q_chi, q_clo, q_sums, k_sums[3], sums_bytes;
+    size_t bis_order, bis_delta, q_chi, q_clo, q_sums, k_sums[3], sums_bytes, lse, vmean;
+    bool comp;
     size_t total;
 };
 
@@ -156,6 +162,9 @@ scope_status check_params(const scope_tensor *q, const scope_grid *g, const scop
         if ((int64_t)g->T * g->Hh * g->W != N) return fail(SCOPE_ESHAPE, "grid: T*Hh*W must equal N");
     }
     if (p->fixed_cluster_size < 0) return fail(SCOPE_EINVAL, "params: fixed_cluster_size must be >= 0");
+    if (p->compensate != 0 && p->compensate != 1) return fail(SCOPE_EINVAL, "params: compensate must be 0 or 1");
+    if (p->compensate && p->fixed_cluster_size == 0)
+        return fail(SCOPE_EINVAL, "params: compensate needs the ClusterAttention variant (fixed_cluster_size > 0)");
     if (p->fixed_cluster_size > 0) {
         const int64_t f = p->fixed_cluster_size;
         if (has_grid) return fail(SCOPE_EINVAL, "fixed_cluster_size needs grid {0,0,0} (no RoPE)");
@@ -238,6 +247,9 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     }
     L.bis_order = take(cur, L.bisect ? 2 * BH * N * 4 : 0);
     L.bis_delta = take(cur, L.bisect ? BH * N * 8 : 0);
+    L.comp = p->compensate != 0;
+    L.lse = take(cur, L.comp ? BH * N * 4 : 0);
+    L.vmean = take(cur, L.comp ? BH * L.C[0] * D * 4 : 0);
     L.k_codes = take(cur, 3 * BH * N * 4);
     for (int s = 0; s < 3; ++s) {
         L.k_cent[s] = take(cur, BH * L.C[s] * (ds[s] > 0 ? ds[s] : 1) * 4);
@@ -513,9 +525,17 @@ extern "C" scope_status scope_attn(const scope_tensor *q, const scope_tensor *k,
     if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
                    at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, at<int32_t>(ws, L.q_sizes),
                    at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start), at<long long>(ws, L.offsets),
-                   at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n), at<int32_t>(ws, L.stats) + 4, (int)L.BH,
-                   (int)L.N, (int)L.D, L.Cq, s))
+                   at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n), at<int32_t>(ws, L.stats) + 4,
+                   L.comp ? at<float>(ws, L.lse) : nullptr, (int)L.BH, (int)L.N, (int)L.D, L.Cq, s))
         return fail(SCOPE_ECUDA, "scope_attn: tensor map encoding failed");
+    if (L.comp)
+        // ClusterAttention: excluded key clusters enter through their mean key and value
+        launch_compensate(at<__nv_bfloat16>(ws, L.qr), vb, at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start),
+                          at<int32_t>(ws, L.k_perm[0]), at<int32_t>(ws, L.k_start[0]), at<int32_t>(ws, L.k_codes),
+                          at<int32_t>(ws, L.k_sizes[0]), at<float>(ws, L.k_cent[0]), at<float>(ws, L.vmean),
+                          at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n),
+                          at<float>(ws, L.lse), (__nv_bfloat16 *)o->ptr, (int)L.BH, (int)L.N, (int)L.D, L.Cq,
+                          L.C[0], s);
     return launch_status("scope_attn");
 }
 
@@ -590,7 +610,8 @@ extern "C" scope_status scope_dense_attn(const scope_tensor *q, const scope_tens
     const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
     if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
                         at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, nullptr, nullptr, nullptr,
-                        nullptr, nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, (int)L.BH, (int)L.N, (int)L.D, 1, s))
+                        nullptr, nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, nullptr, (int)L.BH, (int)L.N,
+                        (int)L.D, 1, s))
         return fail(SCOPE_ECUDA, "scope_dense_attn: tensor map encoding failed");
     return launch_status("scope_dense_attn");
 }

@@ -61,6 +61,8 @@ class Workload:
     # draw their labels independently (objects occupying regions); None = every
     # token draws its own label.
     label_block: Optional[tuple] = None
+    # ClusterAttention variant: compensate excluded key clusters through their mean
+    compensate: int = 0
 
     @property
     def torch_dtype(self):

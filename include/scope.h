@@ -86,7 +86,17 @@ typedef struct {
  *                  d_t == D, d_h == d_w == 0, N == fixed_cluster_size * 2^L;
  *                  queries and keys are each split by balanced recursive
  *                  2-means bisection into N / fixed_cluster_size clusters
- *                  (c_q and c_t are then taken as that count; pass 0 or it). */
+ *                  (c_q and c_t are then taken as that count; pass 0 or it).
+ *   compensate     0 or 1.  1 (ClusterAttention variant only, and at most
+ *                  1024 key clusters): scope_attn adds every excluded key
+ *                  through its key cluster's mean key and mean value
+ *                  ("ClusterAttention: A training-free speedup of
+ *                  bidirectional attention", abstract: compensation of
+ *                  excluded clusters through their mean).  Reading: the
+ *                  m_ck members of key cluster k missing from query cluster
+ *                  c's list add m_ck * e^{q.mu_k/sqrt(D)} to the softmax
+ *                  denominator and that times the mean value to the
+ *                  numerator. */
 typedef struct {
     int32_t d_t, d_h, d_w;
     double theta;
@@ -97,6 +107,7 @@ typedef struct {
     int32_t k_min;
     int32_t online_topk;
     int32_t fixed_cluster_size;
+    int32_t compensate;
 } scope_params;
 
 typedef struct scope_plan_s scope_plan_t; /* opaque host handle */

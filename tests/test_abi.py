@@ -66,6 +66,8 @@ def test_workspace_bytes_counts_list_capacity(L):
     (dict(iters=-1), 1, "iters"),
     (dict(online_topk=2), 1, "online_topk"),
     (dict(fixed_cluster_size=64), 1, "grid"),
+    (dict(compensate=2), 1, "compensate"),
+    (dict(compensate=1), 1, "compensate"),
 ])
 def test_bad_params_rejected_on_host(L, mut, code, msg):
     p, g = P(**mut)

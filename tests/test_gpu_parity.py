@@ -295,3 +295,37 @@ def test_bisection_small_shapes(N, D, H):
     w = synth.WORKLOADS["unstructured"].with_(N=N, D=D, H=H, d_split=(D, 0, 0), components=16, k_min=32,
                                                config_id=150 + N, c_q=N // 64, c_sub=(N // 64, 1, 1))
     bisect_parity(w, range(H))
+
+
+# ClusterAttention compensation: every excluded key enters through its key
+# cluster's mean key and value (the oracle's attention_rows_comp, reading R16),
+# fed the device's own rotated rows, key-cluster labels and lists.
+@pytest.mark.parametrize("N,D,H,p", [(4096, 64, 2, 0.9), (4096, 64, 1, 0.5), (512, 128, 1, 0.9)])
+def test_compensation_parity(N, D, H, p):
+    w = synth.WORKLOADS["unstructured"].with_(N=N, D=D, H=H, d_split=(D, 0, 0), components=16, k_min=32,
+                                               config_id=170 + N + D, c_q=N // 64, c_sub=(N // 64, 1, 1),
+                                               top_p=p, compensate=1)
+    q, k, v = synth.make_inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    pl = plan_of(w, qd, kd)
+    o = scope.attn(qd, kd, vd, pl)
+    pl_plain = plan_of(w.with_(compensate=0), qd, kd)
+    o_plain = scope.attn(qd, kd, vd, pl_plain)
+    torch.cuda.synchronize()
+    pl.sync_status()
+    rng = np.random.default_rng(5)
+    for h in range(H):
+        qr, kr = P.np64(pl.view("qr")[0, h]), P.np64(pl.view("kr")[0, h])
+        vv = v[0, h].double().numpy()
+        qlab = pl.view("q_labels")[0, h].cpu().numpy()
+        klab = pl.view("k_codes")[0, 0, h].cpu().numpy()
+        get = lists_fn(pl, w, h)
+        rows = np.sort(rng.choice(N, 96, replace=False))
+        ref = np.stack([oracle.attention_rows_comp(qr[n:n + 1], kr, vv, get(qlab[n]), klab, 1.0 / np.sqrt(D))[0]
+                        for n in rows])
+        max_abs, rel = P.attn_error(P.np64(o[0, h])[rows], ref)
+        assert max_abs <= P.ATTN_MAX_ABS and rel <= P.ATTN_REL_L2, f"compensated: max-abs {max_abs:.3g}, rel {rel:.3g}"
+        # rows whose cluster kept every key are untouched by the compensation
+        full = [n for n in rows if len(get(qlab[n])) == N]
+        if full:
+            np.testing.assert_array_equal(o[0, h, full].cpu().numpy(), o_plain[0, h, full].cpu().numpy())
