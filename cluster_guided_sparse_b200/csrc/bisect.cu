@@ -23,6 +23,7 @@ namespace scope {
 namespace {
 
 constexpr int kBT = 1024;
+constexpr int kSplitNodes = 64;  // most nodes per head on a split level
 
 __device__ __forceinline__ unsigned long long dkey(double d)
 {
@@ -53,10 +54,18 @@ __device__ void select_k(BisectShared &S, const double *delta, int n, int k, uns
         __syncthreads();
         const unsigned long long pre = S.prefix;
         const int hi = shift + 8;
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const unsigned long long u = dkey(delta[i]);
-            if (hi < 64 && (u >> hi) != (pre >> hi)) continue;
-            atomicAdd(&S.hist[(u >> shift) & 255ull], 1);
+        // A node's deltas share their leading bytes, so most keys fall in one
+        // bucket: add per warp (one atomic per distinct bucket) instead of
+        // per key, which would serialise on that bucket.
+        for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+            const int i = i0 + threadIdx.x;
+            int b = -1;
+            if (i < n) {
+                const unsigned long long u = dkey(delta[i]);
+                if (hi >= 64 || (u >> hi) == (pre >> hi)) b = (int)((u >> shift) & 255ull);
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, b);
+            if (b >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&S.hist[b], __popc(peers));
         }
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -74,6 +83,55 @@ __device__ void select_k(BisectShared &S, const double *delta, int n, int k, uns
     *need = k - S.below;
 }
 
+// delta = ||x - c0||^2 - ||x - c1||^2 in fp64, dims in order.
+__device__ __forceinline__ double split_delta(const __nv_bfloat16 *x, const double *c0, const double *c1, int D)
+{
+    double d0 = 0.0, d1 = 0.0;
+    for (int k = 0; k < D; ++k) {
+        const double xv = (double)__bfloat162float(x[k]);
+        const double t0 = xv - c0[k], t1 = xv - c1[k];
+        d0 = fma(t0, t0, d0);
+        d1 = fma(t1, t1, d1);
+    }
+    return d0 - d1;
+}
+
+// One ordered pass over a node's members: f(i, side0) for every thread and
+// every block of members (i >= n gives side0 = false), where side0 says
+// member i goes to child 0 under (cut, need) -- keys below the cut, then the
+// first `need` members at the cut in member order.  Block-wide.
+template <class F>
+__device__ void each_side(BisectShared &S, const double *delta, int n, unsigned long long cut, int need, F &&f)
+{
+    int eq_run = 0;
+    for (int b0 = 0; b0 < n; b0 += blockDim.x) {
+        const int i = b0 + threadIdx.x;
+        const unsigned long long u = i < n ? dkey(delta[i]) : ~0ull;
+        const int eq = (i < n && u == cut) ? 1 : 0;
+        int tot;
+        const int ex = block_excl_scan(eq, S.tmp, tot);
+        f(i, i < n && (u < cut || (eq && eq_run + ex < need)));
+        eq_run += tot;
+    }
+}
+
+// Stable partition of a node's members by side: child 0 in member order, then child 1.
+__device__ void partition_node(BisectShared &S, const double *delta, int n, unsigned long long cut, int need,
+                               const int32_t *mem, int32_t *out)
+{
+    const int half = n >> 1;
+    int s0_run = 0;
+    each_side(S, delta, n, cut, need, [&](int i, bool side0) {
+        int tot0;
+        const int ex0 = block_excl_scan(side0 ? 1 : 0, S.tmp, tot0);
+        if (i < n) {
+            const int pos0 = s0_run + ex0;
+            out[side0 ? pos0 : half + (i - pos0)] = mem[i];
+        }
+        s0_run += tot0;
+    });
+}
+
 }  // namespace
 
 struct BisectArgs {
@@ -81,6 +139,9 @@ struct BisectArgs {
     int32_t *order;           // [BH][N] members, node by node (in/out)
     int32_t *order_tmp;       // [BH][N]
     double *delta;            // [BH][N]
+    uint8_t *side;            // [BH][N] child of each member (split levels)
+    double *cent;             // [BH][kSplitNodes][2][D] node centroids (split levels)
+    double *gsum;             // [BH][kSplitNodes][2][D] side sums, zero between rounds
     int N, D, level, iters;
 };
 
@@ -90,6 +151,7 @@ __global__ void __launch_bounds__(kBT) bisect_level_kernel(BisectArgs a)
     __shared__ BisectShared S;
     const int node = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int n = a.N >> a.level, D = a.D, half = n >> 1;
+    const int nsl = blockDim.x >> 6;  // member slices of the update (blockDim in 128..1024)
     int32_t *mem = a.order + (int64_t)bh * a.N + (int64_t)node * n;
     int32_t *out = a.order_tmp + (int64_t)bh * a.N + (int64_t)node * n;
     double *delta = a.delta + (int64_t)bh * a.N + (int64_t)node * n;
@@ -104,41 +166,23 @@ __global__ void __launch_bounds__(kBT) bisect_level_kernel(BisectArgs a)
     int need = 0;
     for (int r = 0; r <= a.iters; ++r) {
         // delta of every member
-        for (int i = tid; i < n; i += blockDim.x) {
-            const __nv_bfloat16 *x = X + (int64_t)mem[i] * D;
-            double d0 = 0.0, d1 = 0.0;
-            for (int k = 0; k < D; ++k) {
-                const double xv = (double)__bfloat162float(x[k]);
-                const double t0 = xv - S.c[0][k], t1 = xv - S.c[1][k];
-                d0 = fma(t0, t0, d0);
-                d1 = fma(t1, t1, d1);
-            }
-            delta[i] = d0 - d1;
-        }
+        for (int i = tid; i < n; i += blockDim.x) delta[i] = split_delta(X + (int64_t)mem[i] * D, S.c[0], S.c[1], D);
         __syncthreads();
         select_k(S, delta, n, half, &cut, &need);
         if (r == a.iters) break;
-        // mark sides with one ordered pass (eq keys taken in member order)
-        int eq_run = 0;
-        for (int b0 = 0; b0 < n; b0 += blockDim.x) {
-            const int i = b0 + tid;
-            const unsigned long long u = i < n ? dkey(delta[i]) : ~0ull;
-            const int eq = (i < n && u == cut) ? 1 : 0;
-            int tot;
-            const int ex = block_excl_scan(eq, S.tmp, tot);
-            if (i < n) {
-                const bool side0 = u < cut || (eq && eq_run + ex < need);
-                delta[i] = side0 ? 0.0 : 1.0;  // reuse as the side flag for the sums
-            }
-            eq_run += tot;
-        }
+        // mark sides, reusing delta as the side flag for the sums (a thread
+        // reads and then overwrites only its own member's entry)
+        each_side(S, delta, n, cut, need, [&](int i, bool side0) {
+            if (i < n) delta[i] = side0 ? 0.0 : 1.0;
+        });
         __syncthreads();
-        // update: exact fp64 sums of each side (64 dims x 16 member slices per pass)
+        // update: exact fp64 sums of each side (64 dims x blockDim/64 member
+        // slices per pass; exact, so the slicing does not change the sums)
         for (int d0 = 0; d0 < D; d0 += 64) {
             const int dim = tid & 63, slice = tid >> 6;
             double s0 = 0.0, s1 = 0.0;
             if (d0 + dim < D) {
-                for (int i = slice; i < n; i += 16) {
+                for (int i = slice; i < n; i += nsl) {
                     const double xv = (double)__bfloat162float(X[(int64_t)mem[i] * D + d0 + dim]);
                     if (delta[i] == 0.0) s0 += xv;
                     else s1 += xv;
@@ -151,7 +195,7 @@ __global__ void __launch_bounds__(kBT) bisect_level_kernel(BisectArgs a)
                 const int which = tid >> 6, dd = tid & 63;
                 if (d0 + dd < D) {
                     double sum = 0.0;
-                    for (int q = 0; q < 16; ++q) sum += S.part[which][q][dd];
+                    for (int q = 0; q < nsl; ++q) sum += S.part[which][q][dd];
                     S.c[which][d0 + dd] = sum / (double)half;
                 }
             }
@@ -159,23 +203,107 @@ __global__ void __launch_bounds__(kBT) bisect_level_kernel(BisectArgs a)
         }
     }
     // stable partition by the final cut: side 0 (member order), then side 1
-    int eq_run = 0, s0_run = 0;
-    for (int b0 = 0; b0 < n; b0 += blockDim.x) {
-        const int i = b0 + tid;
-        const unsigned long long u = i < n ? dkey(delta[i]) : ~0ull;
-        const int eq = (i < n && u == cut) ? 1 : 0;
-        int tot;
-        const int ex = block_excl_scan(eq, S.tmp, tot);
-        const bool side0 = i < n && (u < cut || (eq && eq_run + ex < need));
-        int tot0;
-        const int ex0 = block_excl_scan(side0 ? 1 : 0, S.tmp, tot0);
-        if (i < n) {
-            const int pos0 = s0_run + ex0;
-            const int pos = side0 ? pos0 : half + (i - pos0);
-            out[pos] = mem[i];
+    partition_node(S, delta, n, cut, need, mem, out);
+}
+
+// ---------------------------------------------------------------- split levels
+// The top levels have few nodes (one per head at level 0), so one CTA per
+// node would leave most SMs idle.  There each round runs as separate
+// kernels: deltas and side sums over all members of all nodes, the select
+// (and the side marks or the final partition) one CTA per node.  The
+// arithmetic is the fused kernel's: the same fp64 delta, the same select,
+// exact fp64 side sums (now added across CTAs), so the children are the same.
+constexpr int kSplitRows = 256;
+
+__global__ void __launch_bounds__(128) bis_init_kernel(BisectArgs a)
+{
+    const int node = blockIdx.x, bh = blockIdx.y, nodes = gridDim.x;
+    const int n = a.N >> a.level, D = a.D;
+    const int32_t *mem = a.order + (int64_t)bh * a.N + (int64_t)node * n;
+    const __nv_bfloat16 *X = a.X + (int64_t)bh * a.N * D;
+    double *c = a.cent + ((int64_t)bh * nodes + node) * 2 * D;
+    for (int k = threadIdx.x; k < 2 * D; k += blockDim.x) {
+        const int which = k / D, dim = k % D;
+        c[k] = (double)__bfloat162float(X[(int64_t)mem[which ? n >> 1 : 0] * D + dim]);
+    }
+}
+
+__global__ void __launch_bounds__(kSplitRows) bis_delta_kernel(BisectArgs a, int nodes)
+{
+    const int bh = blockIdx.y, D = a.D;
+    const int p = blockIdx.x * kSplitRows + threadIdx.x;
+    if (p >= a.N) return;
+    const int n = a.N >> a.level, node = p / n;
+    const int32_t m = a.order[(int64_t)bh * a.N + p];
+    const double *c = a.cent + ((int64_t)bh * nodes + node) * 2 * D;
+    a.delta[(int64_t)bh * a.N + p] = split_delta(a.X + ((int64_t)bh * a.N + m) * D, c, c + D, D);
+}
+
+// last == 0: mark each member's child; last == 1: write the children.
+__global__ void __launch_bounds__(kBT) bis_select_kernel(BisectArgs a, int last)
+{
+    __shared__ BisectShared S;
+    const int node = blockIdx.x, bh = blockIdx.y;
+    const int n = a.N >> a.level;
+    const int64_t base = (int64_t)bh * a.N + (int64_t)node * n;
+    const double *delta = a.delta + base;
+    unsigned long long cut = 0;
+    int need = 0;
+    select_k(S, delta, n, n >> 1, &cut, &need);
+    if (last) {
+        partition_node(S, delta, n, cut, need, a.order + base, a.order_tmp + base);
+    } else {
+        uint8_t *side = a.side + base;
+        each_side(S, delta, n, cut, need, [&](int i, bool side0) {
+            if (i < n) side[i] = side0 ? 0 : 1;
+        });
+    }
+}
+
+// Side sums of kSplitRows consecutive members (all of one node): 64 dims x
+// kSplitRows/64 member slices per pass, then one fp64 atomic per (side, dim).
+__global__ void __launch_bounds__(kSplitRows) bis_sums_kernel(BisectArgs a, int nodes)
+{
+    __shared__ double part[2][kSplitRows / 64][64];
+    const int bh = blockIdx.y, D = a.D, tid = threadIdx.x;
+    const int p0 = blockIdx.x * kSplitRows;
+    const int n = a.N >> a.level, node = p0 / n;
+    const int32_t *mem = a.order + (int64_t)bh * a.N;
+    const uint8_t *side = a.side + (int64_t)bh * a.N;
+    const __nv_bfloat16 *X = a.X + (int64_t)bh * a.N * D;
+    double *g = a.gsum + ((int64_t)bh * nodes + node) * 2 * D;
+    const int dim = tid & 63, slice = tid >> 6;
+    for (int d0 = 0; d0 < D; d0 += 64) {
+        double s0 = 0.0, s1 = 0.0;
+        if (d0 + dim < D)
+            for (int i = p0 + slice; i < p0 + kSplitRows; i += kSplitRows / 64) {
+                const double xv = (double)__bfloat162float(X[(int64_t)mem[i] * D + d0 + dim]);
+                if (side[i] == 0) s0 += xv;
+                else s1 += xv;
+            }
+        part[0][slice][dim] = s0;
+        part[1][slice][dim] = s1;
+        __syncthreads();
+        if (tid < 128) {
+            const int which = tid >> 6, dd = tid & 63;
+            if (d0 + dd < D) {
+                double sum = 0.0;
+                for (int q = 0; q < kSplitRows / 64; ++q) sum += part[which][q][dd];
+                atomicAdd(g + which * D + d0 + dd, sum);
+            }
         }
-        eq_run += tot;
-        s0_run += tot0;
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(256) bis_means_kernel(BisectArgs a)
+{
+    const int node = blockIdx.x, bh = blockIdx.y, nodes = gridDim.x;
+    const int half = (a.N >> a.level) >> 1;
+    const int64_t o = ((int64_t)bh * nodes + node) * 2 * a.D;
+    for (int k = threadIdx.x; k < 2 * a.D; k += blockDim.x) {
+        a.cent[o + k] = a.gsum[o + k] / (double)half;
+        a.gsum[o + k] = 0.0;
     }
 }
 
@@ -223,10 +351,17 @@ __global__ void iota_kernel(int32_t *order, int N, int64_t total)
     if (i < total) order[i] = (int32_t)(i % N);
 }
 
-// Bisection of every (bh) row set of X into N/leaf leaves.
+// Bytes of the split-level scratch (member sides, node centroids, side sums).
+size_t bisect_aux_bytes(int BH, int N, int D)
+{
+    return (((size_t)BH * N + 255) & ~(size_t)255) + 2 * (size_t)BH * kSplitNodes * 2 * D * sizeof(double);
+}
+
+// Bisection of every (bh) row set of X into N/leaf leaves.  `aux` holds
+// bisect_aux_bytes(BH, N, D) bytes (256-byte aligned).
 void launch_bisect(const __nv_bfloat16 *X, int BH, int N, int D, int leaf, int iters, int32_t *order,
-                   int32_t *order_tmp, double *delta, int32_t *labels, float *cent, float *cn, int32_t *start,
-                   int32_t *sizes, int32_t *perm, cudaStream_t st)
+                   int32_t *order_tmp, double *delta, void *aux, int32_t *labels, float *cent, float *cn,
+                   int32_t *start, int32_t *sizes, int32_t *perm, cudaStream_t st)
 {
     const int64_t total = (int64_t)BH * N;
     iota_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(order, N, total);
@@ -237,14 +372,37 @@ void launch_bisect(const __nv_bfloat16 *X, int BH, int N, int D, int leaf, int i
     a.D = D;
     a.iters = iters;
     a.delta = delta;
+    a.side = (uint8_t *)aux;
+    a.cent = (double *)((char *)aux + (((size_t)BH * N + 255) & ~(size_t)255));
+    a.gsum = a.cent + (size_t)BH * kSplitNodes * 2 * D;
+    cudaMemsetAsync(a.gsum, 0, (size_t)BH * kSplitNodes * 2 * D * sizeof(double), st);
     int32_t *cur = order, *nxt = order_tmp;
     int level = 0;
     for (int n = N; n > leaf; n >>= 1, ++level) {
         a.order = cur;
         a.order_tmp = nxt;
         a.level = level;
-        bisect_level_kernel<<<dim3(1u << level, BH), kBT, 0, st>>>(a);
-        count_launches(1);
+        const int nodes = 1 << level;
+        if (nodes <= kSplitNodes && nodes * BH < 2 * 148 && n >= 2048 && n % kSplitRows == 0) {
+            const dim3 rows((unsigned)(N / kSplitRows), BH), per_node(nodes, BH);
+            bis_init_kernel<<<per_node, 128, 0, st>>>(a);
+            count_launches(1);
+            for (int r = 0; r <= iters; ++r) {
+                bis_delta_kernel<<<rows, kSplitRows, 0, st>>>(a, nodes);
+                bis_select_kernel<<<per_node, kBT, 0, st>>>(a, r == iters ? 1 : 0);
+                count_launches(2);
+                if (r == iters) break;
+                bis_sums_kernel<<<rows, kSplitRows, 0, st>>>(a, nodes);
+                bis_means_kernel<<<per_node, 256, 0, st>>>(a);
+                count_launches(2);
+            }
+        } else {
+            // a CTA as wide as its node (128..1024 threads): deep levels have many
+            // small nodes, and idle threads would only wait at the barriers
+            const int threads = n >= kBT ? kBT : (n > 128 ? (n + 63) & ~63 : 128);
+            bisect_level_kernel<<<dim3(nodes, BH), threads, 0, st>>>(a);
+            count_launches(1);
+        }
         int32_t *t = cur;
         cur = nxt;
         nxt = t;

@@ -22,8 +22,9 @@ cudaError_t km_configure();
 void launch_km_init(const KmBatch &, int, int, int, uint32_t, cudaStream_t);
 void launch_km_assign_direct(const KmBatch &, int, int, int, cudaStream_t);
 void launch_km_sort(const KmBatch &, int, int, cudaStream_t);
-void launch_bisect(const __nv_bfloat16 *, int, int, int, int, int, int32_t *, int32_t *, double *, int32_t *, float *,
-                   float *, int32_t *, int32_t *, int32_t *, cudaStream_t);
+void launch_bisect(const __nv_bfloat16 *, int, int, int, int, int, int32_t *, int32_t *, double *, void *, int32_t *,
+                   float *, float *, int32_t *, int32_t *, int32_t *, cudaStream_t);
+size_t bisect_aux_bytes(int BH, int N, int D);
 cudaError_t km_tc_configure();
 bool launch_km_assign_tc(const KmProblem &, __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, const float *, int32_t *,
                          int32_t *, int32_t *, cudaStream_t);
@@ -87,7 +88,7 @@ struct Layout {
     size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
     size_t lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
-    size_t bis_order, bis_delta, q_chi, q_clo, q_sums, k_sums[3], sums_bytes, lse, vmean;
+    size_t bis_order, bis_delta, bis_aux, q_chi, q_clo, q_sums, k_sums[3], sums_bytes, lse, vmean;
     bool comp;
     size_t total;
 };
@@ -247,6 +248,7 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     }
     L.bis_order = take(cur, L.bisect ? 2 * BH * N * 4 : 0);
     L.bis_delta = take(cur, L.bisect ? BH * N * 8 : 0);
+    L.bis_aux = take(cur, L.bisect ? bisect_aux_bytes((int)BH, (int)N, (int)D) : 0);
     L.comp = p->compensate != 0;
     L.lse = take(cur, L.comp ? BH * N * 4 : 0);
     L.vmean = take(cur, L.comp ? BH * L.C[0] * D * 4 : 0);
@@ -283,7 +285,8 @@ scope_status check_device(cudaStream_t)
     if (cudaGetDevice(&dev) != cudaSuccess) return fail(SCOPE_EDEVICE, "no CUDA device");
     int major = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    if (major != 10) return fail(SCOPE_EDEVICE, "libscope.so is built for sm_100a; device has compute capability %d.x", major);
+    if (major != 10)
+        return fail(SCOPE_EDEVICE, "libscope.so is built for sm_100a; device has compute capability %d.x", major);
     static bool configured[64] = {false};
     if (dev < 64 && !configured[dev]) {
         if (km_configure() != cudaSuccess || attn_tc_configure() != cudaSuccess || km_tc_configure() != cudaSuccess ||
@@ -412,13 +415,13 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
         const int leaf = p->fixed_cluster_size;
         int32_t *ord = at<int32_t>(ws, L.bis_order);
         launch_bisect(at<__nv_bfloat16>(ws, L.qr), BH, N, D, leaf, p->iters, ord, ord + (int64_t)BH * N,
-                      at<double>(ws, L.bis_delta), at<int32_t>(ws, L.q_lab), at<float>(ws, L.q_cent),
-                      at<float>(ws, L.q_cn), at<int32_t>(ws, L.q_start), at<int32_t>(ws, L.q_sizes),
-                      at<int32_t>(ws, L.q_perm), s);
+                      at<double>(ws, L.bis_delta), ws + L.bis_aux, at<int32_t>(ws, L.q_lab),
+                      at<float>(ws, L.q_cent), at<float>(ws, L.q_cn), at<int32_t>(ws, L.q_start),
+                      at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.q_perm), s);
         launch_bisect(at<__nv_bfloat16>(ws, L.kr), BH, N, D, leaf, p->iters, ord, ord + (int64_t)BH * N,
-                      at<double>(ws, L.bis_delta), at<int32_t>(ws, L.k_codes), at<float>(ws, L.k_cent[0]),
-                      at<float>(ws, L.k_cn[0]), at<int32_t>(ws, L.k_start[0]), at<int32_t>(ws, L.k_sizes[0]),
-                      at<int32_t>(ws, L.k_perm[0]), s);
+                      at<double>(ws, L.bis_delta), ws + L.bis_aux, at<int32_t>(ws, L.k_codes),
+                      at<float>(ws, L.k_cent[0]), at<float>(ws, L.k_cn[0]), at<int32_t>(ws, L.k_start[0]),
+                      at<int32_t>(ws, L.k_sizes[0]), at<int32_t>(ws, L.k_perm[0]), s);
         cudaMemsetAsync(at<int32_t>(ws, L.k_codes) + (int64_t)BH * N, 0, (size_t)2 * BH * N * 4, s);
     } else {
     // Key subspaces always, and the queries when they have few clusters, run
@@ -441,9 +444,9 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     auto assign = [&]() {
         if (tc_q) {
             launch_km_assign_direct(keys, BH, N, D, s);
-            tc_ok = tc_ok && launch_km_assign_tc(all.p[3], at<__nv_bfloat16>(ws, L.q_chi), at<__nv_bfloat16>(ws, L.q_clo),
-                                                 BH, N, D, at<float>(ws, L.qnorm), fix_list, fix_count,
-                                                 at<int32_t>(ws, L.stats) + 4, s);
+            tc_ok = tc_ok && launch_km_assign_tc(all.p[3], at<__nv_bfloat16>(ws, L.q_chi),
+                                                 at<__nv_bfloat16>(ws, L.q_clo), BH, N, D, at<float>(ws, L.qnorm),
+                                                 fix_list, fix_count, at<int32_t>(ws, L.stats) + 4, s);
         } else {
             launch_km_assign_direct(all, BH, N, D, s);
         }
@@ -469,7 +472,8 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
                  L.C[2], L.P, L.Pcap, s);
     run_selection(at<float>(ws, L.lut), at<int32_t>(ws, L.k_codes), at<int32_t>(ws, L.item_id),
                   at<int32_t>(ws, L.item_cnt), at<int32_t>(ws, L.item_n), at<uint16_t>(ws, L.key_item), L.Pcap, N,
-                  L.Cq, L.C[0], L.C[1], L.C[2], BH, p->top_p, 1.0f / sqrtf((float)D), p->k_min, at<int32_t>(ws, L.stats) + 4,
+                  L.Cq, L.C[0], L.C[1], L.C[2], BH, p->top_p, 1.0f / sqrtf((float)D), p->k_min,
+                  at<int32_t>(ws, L.stats) + 4,
                   at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.r), at<int32_t>(ws, L.n), at<int32_t>(ws, L.kh),
                   at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, s);
     if ((st = launch_status("selection")) != SCOPE_OK) return st;

@@ -461,9 +461,10 @@ void launch_emit(const SelArgs &a, const int32_t *n_in, const long long *offsets
 }
 
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
-                   const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch, int Cw, int BH, float top_p,
-                   float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes, int32_t *r, int32_t *n,
-                   int32_t *kh, long long *offsets, int32_t *indices, int online, cudaStream_t st)
+                   const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch,
+                   int Cw, int BH, float top_p, float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes,
+                   int32_t *r, int32_t *n, int32_t *kh, long long *offsets, int32_t *indices, int online,
+                   cudaStream_t st)
 {
     SelArgs a;
     a.lut = lut;

@@ -329,3 +329,30 @@ def test_compensation_parity(N, D, H, p):
         full = [n for n in rows if len(get(qlab[n])) == N]
         if full:
             np.testing.assert_array_equal(o[0, h, full].cpu().numpy(), o_plain[0, h, full].cpu().numpy())
+
+
+# B > 1: (batch, head) pairs run through the same kernels; batch 1's selection
+# and attention are checked against the oracle on the device's own stage inputs.
+def test_second_batch_entry_stage_fed():
+    w = synth.WORKLOADS["small"].with_(B=2, config_id=190)
+    q, k, v = synth.make_inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    pl = plan_of(w, qd, kd)
+    o = scope.attn(qd, kd, vd, pl)
+    torch.cuda.synchronize()
+    pl.sync_status()
+    b, N, D = 1, w.N, w.D
+    tc = P.TieCounter()
+    for h in (0, w.H - 1):
+        qr, kr = P.np64(pl.view("qr")[b, h]), P.np64(pl.view("kr")[b, h])
+        qlab = pl.view("q_labels")[b, h].cpu().numpy()
+        codes = [pl.view("k_codes")[s, b, h].cpu().numpy() for s in range(3)]
+        kc = [P.np64(pl.view(n)[b, h]) for n in ("k_cent_t", "k_cent_h", "k_cent_w")]
+        lut = pl.view("lut")[b, h].cpu().numpy()
+        P.check_lut(P.np64(pl.view("q_centroids")[b, h]), kc, w.d_split, lut.astype(np.float64))
+        get = lists_fn(pl, w, h, B=b)
+        P.check_selection(lut, codes, pl.view("q_sizes")[b, h].cpu().numpy(), pl.view("r")[b, h].cpu().numpy(),
+                          pl.view("kh")[b, h].item(), pl.view("n")[b, h].cpu().numpy(), get, w, N, D,
+                          np.arange(w.c_q), tc)
+        P.check_attention(qr, kr, v[b, h].double().numpy(), qlab, get, P.np64(o[b, h]), np.arange(0, N, 7))
+    tc.assert_ok("batch 1 Top-p counts")
