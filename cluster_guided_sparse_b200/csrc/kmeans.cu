@@ -196,20 +196,32 @@ __global__ void __launch_bounds__(256) km_fixup_kernel(KmProblem P, int N, int D
         const float *cent = P.cent + (int64_t)bh * C * dn;
         double best = INFINITY;
         int arg = 0;
-        for (int j = 0; j < C; ++j) {
-            double d = 0.0;
+        // eight centroids per step, so their shuffle reductions overlap
+        constexpr int U = 8;
+        for (int j0 = 0; j0 < C; j0 += U) {
+            double d[U];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (lane + 32 * q < dn) {
-                    const double t = xv[q] - (double)cent[(int64_t)j * dn + lane + 32 * q];
-                    d = fma(t, t, d);
+            for (int u = 0; u < U; ++u) {
+                d[u] = 0.0;
+                if (j0 + u < C) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (lane + 32 * q < dn) {
+                            const double t = xv[q] - (double)cent[(int64_t)(j0 + u) * dn + lane + 32 * q];
+                            d[u] = fma(t, t, d[u]);
+                        }
                 }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-            if (d < best) {
-                best = d;
-                arg = j;
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int u = 0; u < U; ++u) d[u] += __shfl_xor_sync(0xffffffffu, d[u], o);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (j0 + u < C && d[u] < best) {  // ascending j: ties keep the lowest index
+                    best = d[u];
+                    arg = j0 + u;
+                }
         }
         if (lane == 0) P.labels[(int64_t)bh * N + n] = arg;
     }
