@@ -72,7 +72,7 @@ struct Args {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, Args a)
+    attn_tc_kernel(Args a)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzle atoms.
@@ -446,9 +446,6 @@ bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv
                     const int32_t *start, const long long *offsets, const int32_t *indices, const int32_t *n_c,
                     int32_t *err, float *lse, int BH, int N, int D, int Cq, cudaStream_t st)
 {
-    CUtensorMap tmK, tmV;
-    if (!rows_tensor_map(&tmK, kr, (uint64_t)BH * N, D, 1) || !rows_tensor_map(&tmV, v, (uint64_t)BH * N, D, 1))
-        return false;
     tc::tc_items_kernel<<<1, 1024, 0, st>>>(sizes, items, n_items, BH, sizes ? Cq : 1, N);
     count_launches(1);
     tc::Args a;
@@ -469,9 +466,9 @@ bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv
     a.Cq = Cq;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     if (D == 128)
-        tc::attn_tc_kernel<128><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(tmK, tmV, a);
+        tc::attn_tc_kernel<128><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(a);
     else
-        tc::attn_tc_kernel<64><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(tmK, tmV, a);
+        tc::attn_tc_kernel<64><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(a);
     count_launches(1);
     return true;
 }

@@ -62,17 +62,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
                  : "memory");
 }
 
-// Four rows (y0..y3) x 64 bf16 columns starting at column x, 512 bytes.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *tm, int x, int y0, int y1, int y2,
-                                            int y3, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
-        : "memory");
-}
-
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
