@@ -85,3 +85,20 @@ def test_tile_flops_counts_padded_tiles():
     n = torch.tensor([5, 128, 129, 1, 256, 300])
     # Q tiles x key tiles per cluster: 0, 1x1, 1x2, 2x1, 2x2, 3x3
     assert bench.tile_flops(sizes, n, 128) == 4.0 * 128 * 128 * 128 * 18
+
+
+def test_reference_arm_line_has_the_contract_keys(capsys):
+    sys.path.insert(0, ROOT)
+    import argparse
+
+    import bench
+
+    args = argparse.Namespace(workload="tiny", warmup=1, steps=1, gpus=1)
+    bench.run_reference(args, world=1, rank=0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["higher_is_better"] is False and line["value"] > 0
+    for key in ("metric", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "scaling", "dtype", "data", "config"):
+        assert key in line, key
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
