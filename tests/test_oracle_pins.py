@@ -168,6 +168,30 @@ def test_each_key_its_own_centroid_gives_exact_per_query_topp():
 
 
 # ----------------------------------------------------------------------------- Top-p
+def test_order_matches_library_sort_with_ties():
+    # score descending, then key index ascending (ties by the lower index)
+    rng = np.random.default_rng(21)
+    for N in (1, 7, 40):
+        sc = rng.integers(0, 5, N).astype(np.float64)  # many exact ties
+        want = sorted(range(N), key=lambda j: (-sc[j], j))
+        assert oracle.order(sc).tolist() == want
+
+
+def test_prefix_mass_closed_forms():
+    N = 12
+    # equal scores: the first m keys hold exactly m/N of the mass
+    for m in (0, 1, 5, N):
+        assert oracle.prefix_mass(np.zeros(N), m, 0.7) == pytest.approx(m / N, abs=1e-15)
+    rng = np.random.default_rng(22)
+    sc = rng.standard_normal(N)
+    masses = [oracle.prefix_mass(sc, m, 0.5) for m in range(N + 1)]
+    assert masses[0] == 0.0 and masses[-1] == pytest.approx(1.0, abs=1e-15)
+    assert all(b >= a for a, b in zip(masses, masses[1:]))  # prefixes of the order only add mass
+    # the top key alone: its softmax weight, the largest single weight
+    w = np.exp(0.5 * (sc - sc.max()))
+    assert masses[1] == pytest.approx(w.max() / w.sum(), rel=1e-12)
+
+
 def test_topp_brute_force_minimal_set():
     rng = np.random.default_rng(8)
     for trial in range(60):
