@@ -67,10 +67,12 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(
     uint32_t *__restrict__ maxabs, const double2 *__restrict__ tab, int64_t rows, int N, int D,
     int Hh, int W, int dt, int dh, int maxL, int maxP, int use_rope)
 {
-    const int tpr = D >> 3;
+    __shared__ float bmax[8];
+    const int tpr = D >> 3;  // 8 or 16 threads per row (D is 64 or 128)
+    const int sh = D == 128 ? 4 : 3;
     const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t row = gid / tpr;
-    const int c8 = (int)(gid % tpr);
+    const int64_t row = gid >> sh;  // < rows < 2^31
+    const int c8 = (int)(gid & (tpr - 1));
     const bool valid = row < rows;
     float ss = 0.f, mx = 0.f;
     if (valid) {
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(
         // bf16 ulp).  The kernel stays HBM-bound.
         double y[8];
         if (use_rope) {
-            const int n = (int)(row % N);
+            const int n = (int)row % N;
             const int pos3[3] = {n / (Hh * W), (n / W) % Hh, n % W};
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
@@ -114,8 +116,15 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(
     // Row norm over the tpr lanes that share the row (tpr divides 32).
     for (int o = tpr >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (norm2 && valid && c8 == 0) norm2[row] = ss;
+    // max |x| of the block, then one atomic (per-warp atomics on one word
+    // would serialise)
     mx = warp_max(mx);
-    if ((threadIdx.x & 31) == 0) atomicMax(maxabs, __float_as_uint(mx));
+    if ((threadIdx.x & 31) == 0) bmax[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, bmax[w]);
+        atomicMax(maxabs, __float_as_uint(mx));
+    }
 }
 
 void launch_rope_table(double2 *tab, int T, int Hh, int W, int dt, int dh, int dw, double theta,
