@@ -130,3 +130,15 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(scope, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         scope.lib()
+
+
+def test_compensation_workspace_holds_row_lse_and_cluster_means(L):
+    # ClusterAttention shape: N = 4096, 64-token clusters -> 64 key clusters, D = 64
+    w = synth.WORKLOADS["unstructured"].with_(N=4096, D=64, H=2, d_split=(64, 0, 0), c_q=64, c_sub=(64, 1, 1))
+    q = T(N=4096, D=64, H=2)
+    sizes = []
+    for comp in (0, 1):
+        p, g = scope.make_params(w, compensate=comp)
+        sizes.append(L.scope_plan_workspace_bytes(ctypes.byref(q), ctypes.byref(g), ctypes.byref(p)))
+    BH, N, C, D = 2, 4096, 64, 64
+    assert sizes[0] > 0 and sizes[1] >= sizes[0] + BH * N * 4 + BH * C * D * 4
