@@ -1,24 +1,40 @@
 """Benchmark: one SCOPE attention call (scope_plan + scope_attn) per step.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl scope|reference] [--workload NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl scope|reference]
+                    [--workload NAME] [--top-p P] [--compensate]
 
 A step is one pass of the whole hot path -- 3D-RoPE, key-subspace and query
 k-means, lookup tables, hybrid Top-p/Top-k with the online per-head Top-k,
 list emission, sparse attention -- over one synthetic batch of the
-HunyuanVideo-720p-shaped workload (B=1, H=24, N=118800, d=128, bf16), inputs
-resident in HBM (2.2 GB of Q/K/V, far above the 126 MB L2, so no flush is
-needed between steps).  With N GPUs each rank runs its own call (weak
-scaling, no collective on the data path); `value` is ms per call of the whole
-job: the max-over-ranks time of K steps divided by the K*N calls made.
+HunyuanVideo-720p-shaped workload by default (B=1, H=24, N=118800, d=128,
+bf16), inputs resident in HBM (2.2 GB of Q/K/V, far above the 126 MB L2, so
+no flush is needed between steps).
 
---impl reference times the fp64 CPU oracle on a bounded sample of the same
-workload (rank 0 only) and prints its line with "impl": "reference".
+With N GPUs (one process per GPU; started under torch.distributed.run by
+this script itself when the environment has no WORLD_SIZE) one call's heads
+are split round-robin over the ranks (SCOPE has no cross-head term), every
+rank plans and attends over its own heads, and the output heads are
+all-gathered over NCCL inside the step (--no-gather leaves them sharded).
+The timed region is bracketed by a barrier and a device synchronisation on
+every rank, and its time is the max over ranks; `value` = ms per call.
+
+Besides the contract's keys the line reports the plan and attention times,
+this build's own dense attention at the same shape, the fidelity of the
+sparse output against it (relative L2 and PSNR per head), the selected-key
+density per head, and the oracle on a bounded sample of the same workload
+(`cpu_baseline`, rank 0 at N=1, pinned to one core).
+
+--impl reference times the fp64 CPU oracle on the same workload (rank 0 only;
+the whole call for workloads of N <= 4096, else a bounded sample extrapolated
+to the call) and prints its line with "impl": "reference".
 """
 from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -46,10 +62,11 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def attn_traffic(heads: int):
-    """DRAM bytes of one sparse-attention launch, from the committed ncu capture
-    (profiles/attn_tc_traffic.json) scaled from its heads to `heads`; None if the
-    kernel source changed since the capture."""
+def attn_traffic(heads: int, workload: str):
+    """DRAM bytes of one sparse-attention launch over `heads` heads, from the
+    committed ncu capture (profiles/attn_tc_traffic.json), scaled from its
+    heads; None if the kernel source changed since the capture or the capture
+    is of another workload."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "attn_tc_traffic.json")) as f:
@@ -58,7 +75,7 @@ def attn_traffic(heads: int):
             sha = hashlib.sha256(f.read()).hexdigest()
     except Exception:
         return None
-    if sha != rec.get("kernel_source_sha256"):
+    if sha != rec.get("kernel_source_sha256") or rec.get("workload") != workload:
         return None
     return rec["sparse_dram_bytes_per_launch_captured"] * heads / rec["captured_heads"]
 
@@ -121,16 +138,31 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch(n_gpus: int) -> int:
+    """Re-runs this script as n_gpus ranks under torch.distributed.run."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n_gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def dist_setup(n_gpus: int):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"bench.py: --gpus {n_gpus} but WORLD_SIZE={world}")
     if world > 1:
         import datetime
 
         import torch.distributed as dist
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
@@ -143,22 +175,40 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
-    """Max of a per-rank scalar over all ranks (a device tensor under NCCL, a
-    host tensor under gloo)."""
+def _reduce(x: float, world: int, op) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
     dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
     t = torch.tensor([x], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t, op=op)
     return float(t.item())
 
 
-def job_ms_per_call(rank_ms: float, steps: int, world: int) -> float:
-    """Whole-job ms per call: every rank made `steps` calls inside its timed
-    region; the job's time is the slowest rank's."""
-    return max_over_ranks(rank_ms, world) / (steps * world)
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (a device tensor under NCCL, a
+    host tensor under gloo)."""
+    return _reduce(x, world, torch.distributed.ReduceOp.MAX)
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    return _reduce(x, world, torch.distributed.ReduceOp.SUM)
+
+
+def call_ms(rank_ms: float, steps: int, world: int) -> float:
+    """ms per call: every step is one call whose heads are spread over all
+    ranks, so the job's time for `steps` calls is the slowest rank's."""
+    return max_over_ranks(rank_ms, world) / steps
+
+
+def gather_list(x, world: int) -> list:
+    """Every rank's Python object, in rank order."""
+    if world == 1:
+        return [x]
+    import torch.distributed as dist
+    out = [None] * world
+    dist.all_gather_object(out, x)
+    return out
 
 
 def tile_flops(sizes: torch.Tensor, n: torch.Tensor, d: int, bm: int = 128, bn: int = 128,
@@ -173,7 +223,70 @@ def tile_flops(sizes: torch.Tensor, n: torch.Tensor, d: int, bm: int = 128, bn: 
     return 4.0 * d * bm * bn * float((qtiles * ktiles).sum())
 
 
-# --------------------------------------------------------------------------- oracle sample
+def fidelity(o: torch.Tensor, od: torch.Tensor):
+    """Per (batch, head): relative L2 error of the sparse output against the
+    dense one, and PSNR with the dense head's max |o| as the peak."""
+    rel, psnr = [], []
+    for b in range(o.shape[0]):
+        for h in range(o.shape[1]):
+            a, r = o[b, h].float(), od[b, h].float()
+            err = a - r
+            rel.append(float(err.norm() / r.norm().clamp_min(1e-30)))
+            mse = float(err.pow(2).mean())
+            peak = float(r.abs().max())
+            psnr.append(float("inf") if mse == 0 else 10.0 * math.log10(peak * peak / mse))
+    return rel, psnr
+
+
+def cpu_info():
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, os.cpu_count()
+
+
+class PinnedToOneCore:
+    """Runs the enclosed block on one host core (the oracle is single-threaded
+    C; this keeps the OS from spreading it), then restores the affinity."""
+
+    def __enter__(self):
+        self.old = os.sched_getaffinity(0)
+        self.core = min(self.old)
+        os.sched_setaffinity(0, {self.core})
+        return self
+
+    def __exit__(self, *a):
+        os.sched_setaffinity(0, self.old)
+
+
+# --------------------------------------------------------------------------- oracle timing
+def oracle_full(w):
+    """The whole call (every head, every cluster, every query) on the oracle.
+    Returns (ms, description, seconds); input generation is not timed."""
+    import oracle
+
+    t0 = time.perf_counter()
+    p = oracle.Params.of(w)
+    spent = 0.0
+    for b in range(w.B):
+        for h in range(w.H):
+            qh, kh, vh, _ = synth.make_head(w, b, h, 0, synth.grid_field(w))
+            q, k, v = (oracle._round_bf16(x.astype(np.float64)) if w.dtype == "bf16" else x.astype(np.float64)
+                       for x in (qh, kh, vh))
+            s = time.perf_counter()
+            pl = oracle.scope_plan_head(q, k, p)
+            oracle.scope_attn_head(pl["qr"], pl["kr"], v, pl["q_labels"], pl["lists"])
+            spent += time.perf_counter() - s
+    desc = f"whole call of {w.name} on the oracle: every head, cluster and query (1 thread, not extrapolated)"
+    return spent * 1e3, desc, time.perf_counter() - t0
+
+
 def oracle_sample(w, budget_rows=1024, clusters=2, queries=8):
     """Times the fp64 oracle on a bounded slice of head 0 of workload `w` and
     extrapolates to one whole call (all heads, all rows, all clusters).
@@ -191,6 +304,8 @@ def oracle_sample(w, budget_rows=1024, clusters=2, queries=8):
     qr = oracle.rope3d(q, w.grid, w.d_split, w.theta)
     kr = oracle.rope3d(k, w.grid, w.d_split, w.theta)
     tm["rope"] = time.perf_counter() - s
+    if w.fixed_cluster_size > 0:
+        return _oracle_sample_bisect(w, qr, kr, v, tm, t0, clusters, queries)
     offs = np.cumsum((0,) + tuple(w.d_split))
     # key-subspace and query assignment: per-row cost on the sampled rows
     t_assign = 0.0
@@ -200,15 +315,15 @@ def oracle_sample(w, budget_rows=1024, clusters=2, queries=8):
         C = w.c_sub[si]
         cent = kr[np.arange(C) * (N // C), a:b]
         s = time.perf_counter()
-        lab = oracle.kmeans_assign(kr[rows, a:b], cent)
+        oracle.kmeans_assign(kr[rows, a:b], cent)
         t_assign += (time.perf_counter() - s) * N / len(rows) * (I + 1)
         full = oracle.kmeans_assign(kr[:, a:b], cent) if b > a else np.zeros(N, np.int32)
         s = time.perf_counter()
         cent, _ = oracle.kmeans_update(kr[:, a:b], full, cent)
         t_assign += (time.perf_counter() - s) * I
         kcent.append((cent, full))
-        del lab
-    qcent = qr[np.arange(w.c_q) * (N // w.c_q)]
+    C = w.c_q
+    qcent = qr[np.arange(C) * (N // C)]
     s = time.perf_counter()
     oracle.kmeans_assign(qr[rows], qcent)
     t_assign += (time.perf_counter() - s) * N / len(rows) * (I + 1)
@@ -227,7 +342,7 @@ def oracle_sample(w, budget_rows=1024, clusters=2, queries=8):
         sc = oracle.proxy_scores([L[c] for L in luts], [kc[1] for kc in kcent])
         r = oracle.retained_count(sc, w.top_p, w.k_min, scale)
         lists.append(oracle.emit(sc, r))
-    tm["select"] = (time.perf_counter() - s) * w.c_q / clusters
+    tm["select"] = (time.perf_counter() - s) * C / clusters
     s = time.perf_counter()
     for i in range(queries):
         oracle.attention_rows(qr[i:i + 1], kr, v, lists[i % clusters], scale)
@@ -240,37 +355,93 @@ def oracle_sample(w, budget_rows=1024, clusters=2, queries=8):
     return ms, desc, time.perf_counter() - t0
 
 
+def _oracle_sample_bisect(w, qr, kr, v, tm, t0, clusters, queries):
+    """oracle_sample for the ClusterAttention variant: both bisections of
+    head 0 in full, then selection and attention on a sample."""
+    import oracle
+
+    N, D, leaf = w.N, w.D, w.fixed_cluster_size
+    s = time.perf_counter()
+    qlab, qcent, _ = oracle.bisect(qr, leaf, w.iters)
+    klab, kcent, _ = oracle.bisect(kr, leaf, w.iters)
+    tm["bisect"] = time.perf_counter() - s
+    C = N // leaf
+    s = time.perf_counter()
+    L = oracle.lut(qcent, kcent)
+    tm["lut"] = time.perf_counter() - s
+    zeros = np.zeros(N, np.int32)
+    scale = 1.0 / np.sqrt(D)
+    s = time.perf_counter()
+    lists = []
+    for c in range(clusters):
+        sc = oracle.proxy_scores([L[c], np.zeros(1), np.zeros(1)], [klab, zeros, zeros])
+        lists.append(oracle.emit(sc, oracle.retained_count(sc, w.top_p, w.k_min, scale)))
+    tm["select"] = (time.perf_counter() - s) * C / clusters
+    s = time.perf_counter()
+    for i in range(queries):
+        oracle.attention_rows(qr[i:i + 1], kr, v, lists[i % clusters], scale)
+    tm["attn"] = (time.perf_counter() - s) * N / queries
+    ms = sum(tm.values()) * w.H * w.B * 1e3
+    desc = (f"head 0 of {w.name}: full RoPE pass and both bisections, LUT, selection for {clusters} clusters, "
+            f"attention for {queries} queries; extrapolated x clusters, x queries, x {w.B * w.H} heads (1 thread)")
+    return ms, desc, time.perf_counter() - t0
+
+
+def oracle_timed(w, **sample_kw):
+    """(ms, description, seconds) of the oracle on one core: the whole call
+    for small workloads, else the bounded, extrapolated sample."""
+    with PinnedToOneCore():
+        if w.N <= 4096 and w.fixed_cluster_size == 0:
+            return oracle_full(w)
+        return oracle_sample(w, **sample_kw)
+
+
+def workload_of(args):
+    w = synth.WORKLOADS[args.workload]
+    if getattr(args, "top_p", None) is not None:
+        w = w.with_(top_p=args.top_p)
+    if getattr(args, "compensate", False):
+        w = w.with_(compensate=1)
+    return w
+
+
 # --------------------------------------------------------------------------- arms
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     vals = []
-    spent = 0.0
     for i in range(args.warmup + args.steps):
-        ms, desc, sec = oracle_sample(w, budget_rows=256, clusters=1, queries=4)
-        spent += sec
+        ms, desc, _ = oracle_timed(w, budget_rows=256, clusters=1, queries=4)
         if i >= args.warmup:
             vals.append(ms)
     val = statistics.median(vals)
+    model, nproc = cpu_info()
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "ms", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": val, "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "sample": "bounded oracle sample per step, extrapolated"},
-            "cpu_baseline": {"value": val, "unit": "ms", "cores": 1, "kind": "oracle", "sample": desc},
+            "scaling": "strong", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "top_p": w.top_p,
+                       "sample": "whole call" if "not extrapolated" in desc else
+                       "bounded oracle sample per step, extrapolated"},
+            "cpu_baseline": {"value": val, "unit": "ms", "cores": 1, "kind": "oracle", "sample": desc,
+                             "cpu_model": model, "nproc": nproc, "pinned": "one core (sched_setaffinity)"},
             "e2e": {"value": val, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 def run_scope(args, world, rank, local):
     import cluster_guided_sparse_b200 as scope
+    from cluster_guided_sparse_b200 import shard
 
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     dev = torch.device("cuda", local if world > 1 else 0)
-    q, k, v = synth.make_inputs(w)
+    mine = shard.heads_of(w.H, rank, world)
+    gather = world > 1 and not args.no_gather
+    q, k, v = synth.make_inputs(w, heads=mine)
+    wl = w.with_(H=len(mine))  # this rank's share of the call
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     qd, kd, vd = (t.to(dev) for t in (q, k, v))
-    params, grid = scope.make_params(w)
+    params, grid = scope.make_params(wl)
     ws = torch.empty(scope.workspace_bytes(qd, params, grid), dtype=torch.uint8, device=dev)
     o = torch.empty(qd.shape, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -282,11 +453,13 @@ def run_scope(args, world, rank, local):
 
     for _ in range(args.warmup):
         pl = step()
+        if gather:
+            shard.gather_heads(o, w.H)
     torch.cuda.synchronize()
     pl.sync_status()
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     L0 = scope.lib().scope_kernel_launches()
     with ClockSampler(dev.index) as clocks:
         barrier(world)
@@ -300,38 +473,62 @@ def run_scope(args, world, rank, local):
             ev[i][1].record(stream)
             scope.attn(qd, kd, vd, pl, out=o)
             ev[i][2].record(stream)
+            if gather:
+                shard.gather_heads(o, w.H)
+            ev[i][3].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
     launches = scope.lib().scope_kernel_launches() - L0
-    ms_per_call = job_ms_per_call(t0.elapsed_time(t1), args.steps, world)
-    total_ms = ms_per_call * args.steps * world
-    plan_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    call_median_ms = statistics.median(e[0].elapsed_time(e[2]) for e in ev)
+    ms_per_call = call_ms(t0.elapsed_time(t1), args.steps, world)
+    plan_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev), world)
+    attn_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev), world)
+    gather_ms = max_over_ranks(statistics.mean(e[2].elapsed_time(e[3]) for e in ev), world)
+    call_median_ms = max_over_ranks(statistics.median(e[0].elapsed_time(e[3]) for e in ev), world)
 
-    # algorithmic attention flops of one launch: 4 d sum_c |c| n_c
+    # algorithmic attention flops of one launch: 4 d sum_c |c| n_c (this rank's heads)
     sizes = pl.view("q_sizes").to(torch.int64)
     n = pl.view("n").to(torch.int64)
-    pairs = int((sizes * n).sum())
-    attn_flops = 4.0 * w.D * pairs
-    density = pairs / (w.B * w.H * float(w.N) ** 2)
+    head_pairs = (sizes * n).sum(-1).flatten().double()
+    pairs_local = float(head_pairs.sum())
+    attn_flops_local = 4.0 * w.D * pairs_local
+    attn_flops = sum_over_ranks(attn_flops_local, world)
+    density = sum_over_ranks(pairs_local, world) / (w.B * w.H * float(w.N) ** 2)
+    # algorithmic DRAM bytes of one attention launch (this rank's heads): Q, K,
+    # V read once, O written once, every selected-key list read once
+    attn_bytes_local = 4.0 * qd.numel() * qd.element_size() + 4.0 * float(n.sum())
     hbm, bf16, bf16_sus, src = peaks()
-    achieved = attn_flops / (attn_ms * 1e-3) / 1e12
-    tile_tf = tile_flops(sizes.flatten(), n.flatten(), w.D) / (attn_ms * 1e-3) / 1e12
+    # per-GPU roofline of the attention kernel: this rank's flops over its own launch time
+    attn_ms_local = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    achieved = attn_flops_local / (attn_ms_local * 1e-3) / 1e12
+    achieved = sum_over_ranks(achieved, world) / world
+    tile_tf = sum_over_ranks(tile_flops(sizes.flatten(), n.flatten(), w.D) / (attn_ms_local * 1e-3) / 1e12,
+                             world) / world
 
-    # this build's dense attention (RoPE + all keys) at the same shape, for context
+    # this build's dense attention (RoPE + all keys) on the same heads, and
+    # the fidelity of the sparse output against it
     od = torch.empty_like(o)
     dense = []
     for i in range(1 + args.steps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
         a.record(stream)
         scope.dense_attn(qd, kd, vd, params, grid, out=od)
         b.record(stream)
         torch.cuda.synchronize()
         if i > 0:
             dense.append(a.elapsed_time(b))
-    dense_ms = statistics.mean(dense)
+    dense_ms = max_over_ranks(statistics.mean(dense), world)
+    rel, psnr = fidelity(o, od)
+    dens_heads = (head_pairs / float(w.N) ** 2).tolist()
+    per_rank = gather_list({"heads": mine, "rel": rel, "psnr": psnr, "density": dens_heads}, world)
+    by_head = {}
+    for r in per_rank:
+        for i, h in enumerate(r["heads"]):
+            by_head[h] = (r["rel"][i], r["psnr"][i], r["density"][i])
+    rel_h = [by_head[h][0] for h in range(w.H)]
+    psnr_h = [by_head[h][1] for h in range(w.H)]
+    dens_h = [by_head[h][2] for h in range(w.H)]
     del od
 
     # end to end through the public API with host buffers: Q and K go first
@@ -361,34 +558,50 @@ def run_scope(args, world, rank, local):
         torch.cuda.synchronize()
         if i >= args.warmup:
             e2e.append(a.elapsed_time(b))
-    e2e_ms = max_over_ranks(statistics.mean(e2e), world) / world
-    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
-    d2h = oh.numel() * oh.element_size()
+    e2e_ms = max_over_ranks(statistics.mean(e2e), world)
+    h2d = sum_over_ranks(sum(t.numel() * t.element_size() for t in (qh, kh, vh)), world)
+    d2h = sum_over_ranks(oh.numel() * oh.element_size(), world)
+    launches = int(sum_over_ranks(launches, world))
+    clk = clocks.summary()
 
     if rank != 0:
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        ms, desc, _ = oracle_sample(w)
-        cpu = {"value": ms, "unit": "ms", "cores": 1, "kind": "oracle", "sample": desc}
+        ms, desc, _ = oracle_timed(w)
+        model, nproc = cpu_info()
+        cpu = {"value": ms, "unit": "ms", "cores": 1, "kind": "oracle", "sample": desc, "cpu_model": model,
+               "nproc": nproc, "pinned": "one core (sched_setaffinity)"}
     eff = w.dense_flops() / (ms_per_call * 1e-3) / 1e12
+    traffic = attn_traffic(len(mine) * w.B, args.workload)
+    psnr_fin = [p for p in psnr_h if math.isfinite(p)]
     line = {
         "metric": METRIC, "value": ms_per_call, "unit": "ms", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.N, "heads": w.H,
-                   "head_dim": w.D, "top_p": w.top_p, "online_topk": bool(w.online_topk),
-                   "l2": "inputs 2.2 GB >> 126 MB L2, no flush", "parallelism": f"replicas x{world}"},
-        "effective_tflops": eff, "plan_ms": plan_ms, "attn_ms": attn_ms, "call_median_ms": call_median_ms,
-        "density": density, "tile_tflops": tile_tf, "tile_frac_of_sustained": tile_tf / bf16_sus,
+        "warmup": args.warmup, "ms_per_step": ms_per_call, "higher_is_better": False,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.N, "heads": w.H, "head_dim": w.D,
+                   "top_p": w.top_p, "online_topk": bool(w.online_topk), "compensate": bool(w.compensate),
+                   "l2": f"inputs {3 * w.B * w.H * w.N * w.D * 2 / 1e9:.2g} GB vs 126 MB L2, no flush",
+                   "parallelism": "single GPU" if world == 1 else
+                   f"heads round-robin over {world} GPUs" + (", O all-gathered" if gather else "")},
+        "effective_tflops": eff, "plan_ms": plan_ms, "attn_ms": attn_ms, "gather_ms": gather_ms,
+        "call_median_ms": call_median_ms,
+        "density": density, "density_per_head": [round(x, 4) for x in dens_h],
+        "fidelity_vs_own_dense": {"rel_l2_mean": statistics.mean(rel_h), "rel_l2_max": max(rel_h),
+                                  "psnr_db_mean": statistics.mean(psnr_fin) if psnr_fin else None,
+                                  "psnr_db_min": min(psnr_h), "rel_l2_per_head": [round(x, 5) for x in rel_h],
+                                  "psnr_db_per_head": [round(x, 2) for x in psnr_h]},
+        "tile_tflops": tile_tf, "tile_frac_of_sustained": tile_tf / bf16_sus,
         "own_dense_ms": dense_ms, "speedup_vs_own_dense": dense_ms / ms_per_call,
-        "roofline": {"kernel": "sparse attention (scope_attn)", "bound": "tensor", "achieved": achieved,
-                     "peak": bf16_sus, "unit": "TFLOP/s", "frac": achieved / bf16_sus,
-                     "traffic": attn_traffic(w.B * w.H),
-                     "peak_source": f"{src} bf16 sustained"},
-        "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"kernel": "sparse attention (scope_attn, attn_tc_kernel)", "bound": "tensor",
+                     "achieved": achieved, "peak": bf16_sus, "unit": "TFLOP/s", "frac": achieved / bf16_sus,
+                     "traffic": traffic,
+                     "algorithmic_bytes": attn_bytes_local,
+                     "traffic_over_algorithmic": None if traffic is None else traffic / attn_bytes_local,
+                     "peak_source": f"{src} bf16 sustained", "algorithmic_tflop_per_call": attn_flops / 1e12},
+        "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": launches,
-        "clocks": clocks.summary(),
+        "clocks": clk,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -401,8 +614,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="scope", choices=["scope", "reference"])
     ap.add_argument("--workload", default="hunyuan720p", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--top-p", type=float, default=None, help="override the workload's Top-p")
+    ap.add_argument("--compensate", action="store_true", help="ClusterAttention compensation (unstructured only)")
+    ap.add_argument("--no-gather", action="store_true", help="N > 1: leave the output heads sharded")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args.gpus))
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -32,7 +32,7 @@ _TORCH_DT = {SCOPE_F32: torch.float32, SCOPE_BF16: torch.bfloat16, SCOPE_I32: to
 
 class ScopeTensor(ctypes.Structure):
     _fields_ = [("ptr", ctypes.c_void_p), ("dtype", ctypes.c_int), ("B", ctypes.c_int64), ("H", ctypes.c_int64),
-                ("N", ctypes.c_int64), ("D", ctypes.c_int64)]
+                ("N", ctypes.c_int64), ("D", ctypes.c_int64), ("strides", ctypes.c_int64 * 4)]
 
 
 class ScopeGrid(ctypes.Structure):
@@ -88,7 +88,9 @@ def lib() -> ctypes.CDLL:
         L.scope_plan_destroy.restype = None
         L.scope_last_error.restype = ctypes.c_char_p
         L.scope_version.restype = ctypes.c_int
-        for name in ("scope_plan", "scope_attn", "scope_dense_attn", "scope_plan_view", "scope_sync_status"):
+        L.scope_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+        for name in ("scope_plan", "scope_attn", "scope_dense_attn", "scope_plan_view", "scope_sync_status",
+                     "scope_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -106,22 +108,22 @@ def _check(status: int):
         raise ScopeError(status, lib().scope_last_error().decode())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, device=None) -> ctypes.c_void_p:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
 
 
 def as_tensor(x: torch.Tensor) -> ScopeTensor:
+    """scope_tensor of a [B, H, N, D] tensor with its element strides (the
+    library checks them: last stride 1, 16-byte aligned rows, no overlap)."""
     if x.dim() != 4:
         raise ValueError("expected a [B, H, N, D] tensor")
-    if not x.is_contiguous():
-        raise ValueError("tensor must be contiguous")
     dt = {torch.float32: SCOPE_F32, torch.bfloat16: SCOPE_BF16}.get(x.dtype)
     if dt is None:
         raise ValueError(f"unsupported dtype {x.dtype}")
     B, H, N, D = x.shape
-    return ScopeTensor(x.data_ptr(), dt, B, H, N, D)
+    return ScopeTensor(x.data_ptr(), dt, B, H, N, D, (ctypes.c_int64 * 4)(*x.stride()))
 
 
 def make_params(w=None, **kw):
@@ -163,6 +165,12 @@ class Plan:
     def sync_status(self, stream=None):
         _check(lib().scope_sync_status(self._h, _stream(stream)))
 
+    def selftest_wait_timeout(self, cycles: int = 2_000_000, stream=None):
+        """Enqueue the library's failure-handling self-test: a bounded wait on a
+        barrier nothing completes, which sets this plan's timeout bit (the next
+        sync_status raises ScopeError with SCOPE_ETIMEOUT)."""
+        _check(lib().scope_selftest_wait_timeout(self._h, int(cycles), _stream(stream)))
+
     def __del__(self):
         if getattr(self, "_h", None) and _lib is not None:
             _lib.scope_plan_destroy(self._h)
@@ -184,9 +192,10 @@ def plan(q: torch.Tensor, k: torch.Tensor, params: ScopeParams, grid: ScopeGrid,
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     h = ctypes.c_void_p()
-    _check(lib().scope_plan(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(grid), ctypes.byref(params),
-                            ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream),
-                            ctypes.byref(h)))
+    with torch.cuda.device(q.device):
+        _check(lib().scope_plan(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(grid), ctypes.byref(params),
+                                ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream, q.device),
+                                ctypes.byref(h)))
     return Plan(h, workspace, q, k)
 
 
@@ -195,8 +204,9 @@ def attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, p: Plan, out: Option
     """Step 5 on the device: bf16 [B, H, N, D] attention output."""
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
-    _check(lib().scope_attn(ctypes.byref(as_tensor(q)), ctypes.byref(as_tensor(k)), ctypes.byref(as_tensor(v)),
-                            p._h, ctypes.byref(as_tensor(out)), _stream(stream)))
+    with torch.cuda.device(q.device):
+        _check(lib().scope_attn(ctypes.byref(as_tensor(q)), ctypes.byref(as_tensor(k)), ctypes.byref(as_tensor(v)),
+                                p._h, ctypes.byref(as_tensor(out)), _stream(stream, q.device)))
     return out
 
 
@@ -212,9 +222,11 @@ def dense_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, params: ScopeP
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
-    _check(lib().scope_dense_attn(ctypes.byref(tq), ctypes.byref(as_tensor(k)), ctypes.byref(as_tensor(v)),
-                                  ctypes.byref(grid), ctypes.byref(params), ctypes.byref(as_tensor(out)),
-                                  ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)))
+    with torch.cuda.device(q.device):
+        _check(lib().scope_dense_attn(ctypes.byref(tq), ctypes.byref(as_tensor(k)), ctypes.byref(as_tensor(v)),
+                                      ctypes.byref(grid), ctypes.byref(params), ctypes.byref(as_tensor(out)),
+                                      ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                      _stream(stream, q.device)))
     return out
 
 
@@ -229,11 +241,20 @@ def kmeans_noalloc(x: torch.Tensor, dim_off: int, dim_n: int, C: int, iters: int
     f.argtypes = [ctypes.POINTER(ScopeTensor), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                   ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     f.restype = ctypes.c_int
+    if not x.is_cuda or x.dim() != 4 or x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 [B, H, N, D] CUDA tensor")
     B, H, N, _ = x.shape
     if labels is None:
         labels = torch.empty((B, H, N), dtype=torch.int32, device=x.device)
     if centroids is None:
         centroids = torch.empty((B, H, C, dim_n), dtype=torch.float32, device=x.device)
-    _check(f(ctypes.byref(as_tensor(x)), dim_off, dim_n, C, iters, seed & 0xFFFFFFFF,
-             ctypes.c_void_p(labels.data_ptr()), ctypes.c_void_p(centroids.data_ptr()), _stream(stream)))
+    # the library writes B*H*N labels and B*H*C*dim_n centroids through raw pointers
+    for t, dt, shape, name in ((labels, torch.int32, (B, H, N), "labels"),
+                               (centroids, torch.float32, (B, H, C, dim_n), "centroids")):
+        if t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous() or t.device != x.device:
+            raise ValueError(f"{name} must be a contiguous {dt} tensor of shape {shape} on {x.device}")
+    with torch.cuda.device(x.device):
+        _check(f(ctypes.byref(as_tensor(x)), dim_off, dim_n, C, iters, seed & 0xFFFFFFFF,
+                 ctypes.c_void_p(labels.data_ptr()), ctypes.c_void_p(centroids.data_ptr()),
+                 _stream(stream, x.device)))
     return labels, centroids

@@ -57,6 +57,7 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c, int rows)
 struct Args {
     const __nv_bfloat16 *qr, *kr, *v;
     __nv_bfloat16 *o;
+    RowStrides vs, os;         // caller's V and O rows
     const int4 *items;         // (bh, cluster, first query, query count) per work item
     const int32_t *n_items;    // total work items
     const int32_t *perm;       // [BH][N] or null (dense: identity)
@@ -95,6 +96,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bh = it.x, c = it.y, q0 = it.z, nq = it.w;
     const bool two = nq > BM;
     const int64_t base = (int64_t)bh * a.N;
+    const __nv_bfloat16 *vbh = a.v + a.vs.bh_off(bh);
+    const int64_t vsn = a.vs.sN;
     const int cstart = a.start ? a.start[(int64_t)bh * (a.Cq + 1) + c] : 0;
     const long long loff = a.indices ? a.offsets[(int64_t)bh * a.Cq + c] : 0;
     const int nk = a.indices ? a.n_c[(int64_t)bh * a.Cq + c] : a.N;
@@ -157,16 +160,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 keys[i] = a.indices ? a.indices[loff + kj] : kj;
             }
         };
-        auto issue = [&](unsigned char *dst_base, const __nv_bfloat16 *src, int j) {
+        auto issue = [&](unsigned char *dst_base, const __nv_bfloat16 *src, int64_t sn, int j) {
             const uint32_t dst = smem_u32(dst_base + (j & 1) * KV_BYTES);
 #pragma unroll
             for (int i = 0; i < NR; ++i)
-                cp_async16(dst + sw_off(i * RPI + r0, ch, BN), src + (base + keys[i]) * D + ch * 8, true);
+                cp_async16(dst + sw_off(i * RPI + r0, ch, BN), src + keys[i] * sn + ch * 8, true);
             cp_async_commit();
         };
+        const __nv_bfloat16 *kbh = a.kr + base * D;
         load_keys(0);
-        issue(sK, a.kr, 0);
-        issue(sV, a.v, 0);
+        issue(sK, kbh, D, 0);
+        issue(sV, vbh, vsn, 0);
         for (int j = 0; j < ntiles; ++j) {
             const bool more = j + 1 < ntiles;
             // in flight: K(j), V(j)
@@ -179,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j + 1 >= 2 && !mbar_wait(&bar_k_empty[(j + 1) & 1], (((j + 1) >> 1) - 1) & 1, abort_flag, a.err,
                                              0x10))
                     break;
-                issue(sK, a.kr, j + 1);
+                issue(sK, kbh, D, j + 1);
                 cp_async_wait1();  // in flight: V(j), K(j+1)
             } else {
                 cp_async_wait_all();
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j + 1 >= 2 && !mbar_wait(&bar_v_empty[(j + 1) & 1], (((j + 1) >> 1) - 1) & 1, abort_flag, a.err,
                                              0x11))
                     break;
-                issue(sV, a.v, j + 1);
+                issue(sV, vbh, vsn, j + 1);
             }
         }
         cp_async_wait_all();
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float inv = 1.f / l;
             // row log-sum-exp, natural log: the row's exponentials are 2^(s*scale*log2e - m_run)
             if (a.lse && store) a.lse[base + tok] = (m_run + log2f(l)) * 0.6931471805599453f;
-            __nv_bfloat16 *dst = a.o + (base + tok) * D;
+            __nv_bfloat16 *dst = a.o + a.os.row(bh, tok);
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t o[32];
@@ -441,8 +445,8 @@ bool rows_tensor_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv_bfloat16 *v, __nv_bfloat16 *o,
-                    int4 *items, int32_t *n_items, int max_items, const int32_t *sizes, const int32_t *perm,
+bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv_bfloat16 *v, const RowStrides &vs,
+                    __nv_bfloat16 *o, const RowStrides &os, int4 *items, int32_t *n_items, int max_items, const int32_t *sizes, const int32_t *perm,
                     const int32_t *start, const long long *offsets, const int32_t *indices, const int32_t *n_c,
                     int32_t *err, float *lse, int BH, int N, int D, int Cq, cudaStream_t st)
 {
@@ -453,6 +457,8 @@ bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv
     a.kr = kr;
     a.v = v;
     a.o = o;
+    a.vs = vs;
+    a.os = os;
     a.items = items;
     a.n_items = n_items;
     a.perm = perm;

@@ -11,6 +11,7 @@ constexpr int kSortBlk = 512;   // points per warp-block in the stable label sor
 constexpr int kMaxClusters = 1024;
 constexpr int kTQ = 128;        // query rows per attention tile
 constexpr int kMaxItems = 65536; // c_t * c_h * c_w bound (distinct code triples)
+constexpr int kScanTileCounters = 4096;  // block counters per tile of the label-sort scan
 
 // Device error word bits (workspace int32[4]).
 constexpr int kErrRange = 1;
@@ -20,7 +21,7 @@ constexpr int kErrTimeout = 2;
 // clusters.  Key subspaces and queries of one plan run as one batch.
 struct KmProblem {
     const __nv_bfloat16 *X;     // [BH][N][D]
-    const uint32_t *maxabs;     // bits of max |X| (non-negative float), set by RoPE
+    const uint32_t *maxabs;     // [BH] bits of max |X| per (batch, head) (non-negative float), set by RoPE
     int dim_off, dim_n, C;
     int32_t *labels;            // [BH][N]
     float *cent;                // [BH][C][dim_n]
@@ -29,7 +30,18 @@ struct KmProblem {
     int32_t *perm;              // [BH][N]   members cluster by cluster, ascending
     int32_t *start;             // [BH][C+1] cluster starts in perm
     int32_t *blockhist;         // [BH][C][nblk]
+    int32_t *tilesum;           // [BH][ceil(C*nblk / 4096)] scan tile sums
     unsigned long long *sums;   // [BH][C][dim_n] fixed-point member sums, zero between updates (or null)
+};
+
+// Where the rows of a caller's [B, H, N, D] tensor live: row (b, h, n)
+// starts at element b*sB + h*sH + n*sN (D contiguous elements).  Kernels index
+// by the flat (batch, head) number bh = b*H + h.
+struct RowStrides {
+    int64_t sB, sH, sN;
+    int H;
+    __host__ __device__ __forceinline__ int64_t bh_off(int64_t bh) const { return (bh / H) * sB + (bh % H) * sH; }
+    __host__ __device__ __forceinline__ int64_t row(int64_t bh, int64_t n) const { return bh_off(bh) + n * sN; }
 };
 
 struct KmBatch {

@@ -23,17 +23,17 @@ constexpr int kCompThreads = 128;
 
 // vbar_k: mean of V over the members of key cluster k (fp64 sums), one
 // thread per dim.
-__global__ void vmean_kernel(const __nv_bfloat16 *V, const int32_t *perm, const int32_t *start, float *vmean, int N,
-                             int D, int C)
+__global__ void vmean_kernel(const __nv_bfloat16 *V, RowStrides vs, const int32_t *perm, const int32_t *start,
+                             float *vmean, int N, int D, int C)
 {
     const int k = blockIdx.x, bh = blockIdx.y, d = threadIdx.x;
     if (d >= D) return;
     const int32_t *st = start + (int64_t)bh * (C + 1);
     const int s0 = st[k], s1 = st[k + 1];
     const int32_t *pm = perm + (int64_t)bh * N;
-    const __nv_bfloat16 *Vb = V + (int64_t)bh * N * D;
+    const __nv_bfloat16 *Vb = V + vs.bh_off(bh);
     double acc = 0.0;
-    for (int t = s0; t < s1; ++t) acc += (double)__bfloat162float(Vb[(int64_t)pm[t] * D + d]);
+    for (int t = s0; t < s1; ++t) acc += (double)__bfloat162float(Vb[(int64_t)pm[t] * vs.sN + d]);
     vmean[((int64_t)bh * C + k) * D + d] = s1 > s0 ? (float)(acc / (double)(s1 - s0)) : 0.f;
 }
 
@@ -49,7 +49,8 @@ struct CompArgs {
     const int32_t *indices;      // selected-key lists
     const int32_t *n_c;          // [BH][Cq]
     const float *lse;            // [BH][N] log-sum-exp of the attention rows
-    __nv_bfloat16 *o;            // [BH][N][D] in: o_S, out: compensated
+    __nv_bfloat16 *o;            // caller's rows (strides os) in: o_S, out: compensated
+    RowStrides os;
     int N, Cq, Ck;
     float scale;                 // 1 / sqrt(D)
 };
@@ -98,11 +99,12 @@ __global__ void __launch_bounds__(kCompThreads) comp_kernel(CompArgs a)
     for (int r = q0 + threadIdx.x; r < q1; r += blockDim.x) {
         const int tok = a.q_perm[(int64_t)bh * a.N + r];
         const int64_t row = (int64_t)bh * a.N + tok;
+        __nv_bfloat16 *orow = a.o + a.os.row(bh, tok);
         float q[D], acc[D];
 #pragma unroll
         for (int d = 0; d < D; ++d) {
             q[d] = __bfloat162float(a.qr[row * D + d]) * a.scale;
-            acc[d] = __bfloat162float(a.o[row * D + d]);
+            acc[d] = __bfloat162float(orow[d]);
         }
         float mx = a.lse[row], den = 1.f;  // the selected keys: weight e^{L_S}, value o_S
         for (int e = 0; e < n_ex; ++e) {
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(kCompThreads) comp_kernel(CompArgs a)
 #pragma unroll
         for (int d = 0; d < D; d += 2) {
             __nv_bfloat162 h = __floats2bfloat162_rn(acc[d] * inv, acc[d + 1] * inv);
-            *reinterpret_cast<__nv_bfloat162 *>(a.o + row * D + d) = h;
+            *reinterpret_cast<__nv_bfloat162 *>(orow + d) = h;
         }
     }
 }
@@ -138,13 +140,13 @@ __global__ void __launch_bounds__(kCompThreads) comp_kernel(CompArgs a)
 }  // namespace
 
 // Mean values of the key clusters, then the compensation of every query row.
-void launch_compensate(const __nv_bfloat16 *qr, const __nv_bfloat16 *v, const int32_t *q_perm,
+void launch_compensate(const __nv_bfloat16 *qr, const __nv_bfloat16 *v, const RowStrides &vs, const int32_t *q_perm,
                        const int32_t *q_start, const int32_t *k_perm, const int32_t *k_start, const int32_t *klab,
                        const int32_t *ksize, const float *kcent, float *vmean, const long long *offsets,
-                       const int32_t *indices, const int32_t *n_c, const float *lse, __nv_bfloat16 *o, int BH, int N,
-                       int D, int Cq, int Ck, cudaStream_t st)
+                       const int32_t *indices, const int32_t *n_c, const float *lse, __nv_bfloat16 *o,
+                       const RowStrides &os, int BH, int N, int D, int Cq, int Ck, cudaStream_t st)
 {
-    vmean_kernel<<<dim3(Ck, BH), D, 0, st>>>(v, k_perm, k_start, vmean, N, D, Ck);
+    vmean_kernel<<<dim3(Ck, BH), D, 0, st>>>(v, vs, k_perm, k_start, vmean, N, D, Ck);
     count_launches(1);
     CompArgs a;
     a.qr = qr;
@@ -159,6 +161,7 @@ void launch_compensate(const __nv_bfloat16 *qr, const __nv_bfloat16 *v, const in
     a.n_c = n_c;
     a.lse = lse;
     a.o = o;
+    a.os = os;
     a.N = N;
     a.Cq = Cq;
     a.Ck = Ck;

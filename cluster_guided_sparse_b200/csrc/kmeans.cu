@@ -178,15 +178,21 @@ static size_t direct_smem(int dn)
 // The tensor-core query assignment (kmeans_tc.cu) lists the rows whose best
 // and second-best expanded-form scores lie within its fp32 error margin.
 // Exact re-decision of the listed rows: fp64 direct-form distance to every
-// centroid, lowest index on ties.  One warp per row.
-__global__ void __launch_bounds__(256) km_fixup_kernel(KmProblem P, int N, int D, const int32_t *fix_list,
-                                                       const int32_t *fix_count)
+// centroid, lowest index on ties.  One CTA per listed row (grid-strided):
+// warp w takes centroids w, w + 8, ..., its lanes split the dims, and eight
+// centroids per step keep eight shuffle reductions in flight; the eight
+// warps' winners then meet in shared memory.
+constexpr int kFixWarps = 8;
+
+__global__ void __launch_bounds__(kFixWarps * 32) km_fixup_kernel(KmProblem P, int N, int D, const int32_t *fix_list,
+                                                                  const int32_t *fix_count)
 {
-    const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (blockDim.x >> 5);
+    __shared__ double wbest[kFixWarps];
+    __shared__ int warg[kFixWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int count = *fix_count;
     const int C = P.C, dn = P.dim_n;
-    for (int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < count; w += warps) {
+    for (int w = blockIdx.x; w < count; w += gridDim.x) {
         const int gid = fix_list[w];
         const int bh = gid / N, n = gid % N;
         const __nv_bfloat16 *x = P.X + ((int64_t)bh * N + n) * D + P.dim_off;
@@ -195,19 +201,19 @@ __global__ void __launch_bounds__(256) km_fixup_kernel(KmProblem P, int N, int D
         for (int q = 0; q < 4; ++q) xv[q] = lane + 32 * q < dn ? (double)__bfloat162float(x[lane + 32 * q]) : 0.0;
         const float *cent = P.cent + (int64_t)bh * C * dn;
         double best = INFINITY;
-        int arg = 0;
-        // eight centroids per step, so their shuffle reductions overlap
+        int arg = C;
         constexpr int U = 8;
-        for (int j0 = 0; j0 < C; j0 += U) {
+        for (int j0 = warp; j0 < C; j0 += U * kFixWarps) {
             double d[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 d[u] = 0.0;
-                if (j0 + u < C) {
+                const int j = j0 + u * kFixWarps;
+                if (j < C) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         if (lane + 32 * q < dn) {
-                            const double t = xv[q] - (double)cent[(int64_t)(j0 + u) * dn + lane + 32 * q];
+                            const double t = xv[q] - (double)cent[(int64_t)j * dn + lane + 32 * q];
                             d[u] = fma(t, t, d[u]);
                         }
                 }
@@ -217,13 +223,30 @@ __global__ void __launch_bounds__(256) km_fixup_kernel(KmProblem P, int N, int D
 #pragma unroll
                 for (int u = 0; u < U; ++u) d[u] += __shfl_xor_sync(0xffffffffu, d[u], o);
 #pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (j0 + u < C && d[u] < best) {  // ascending j: ties keep the lowest index
+            for (int u = 0; u < U; ++u) {
+                const int j = j0 + u * kFixWarps;  // ascending within the warp: ties keep the lowest index
+                if (j < C && d[u] < best) {
                     best = d[u];
-                    arg = j0 + u;
+                    arg = j;
                 }
+            }
         }
-        if (lane == 0) P.labels[(int64_t)bh * N + n] = arg;
+        if (lane == 0) {
+            wbest[warp] = best;
+            warg[warp] = arg;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double b = wbest[0];
+            int a = warg[0];
+            for (int i = 1; i < kFixWarps; ++i)
+                if (wbest[i] < b || (wbest[i] == b && warg[i] < a)) {
+                    b = wbest[i];
+                    a = warg[i];
+                }
+            P.labels[(int64_t)bh * N + n] = a;
+        }
+        __syncthreads();
     }
 }
 
@@ -246,29 +269,81 @@ __global__ void km_hist_kernel(KmBatch b, int N, int nblk)
     for (int c = lane; c < P.C; c += 32) h[(int64_t)c * nblk + blk] = hist[c];
 }
 
-// Exclusive scan over (cluster, block) -> stable output bases; cluster starts.
-__global__ void __launch_bounds__(1024) km_scan_kernel(KmBatch b, int N, int nblk)
+// Exclusive scan over (cluster, block) -> stable output bases; cluster starts
+// and sizes.  Three parallel steps per (head, problem): the sums of tiles of
+// kScanTile counters, then every tile scans its counters from the sum of the
+// tiles before it (so no CTA walks C x blocks counters alone), then the
+// cluster starts and sizes.
+constexpr int kScanThreads = 1024, kScanPer = 4, kScanTile = kScanThreads * kScanPer;
+static_assert(kScanTile == kScanTileCounters, "scan tile size");
+
+__global__ void __launch_bounds__(kScanThreads) km_scan_tiles_kernel(KmBatch b, int nblk)
 {
     __shared__ int tmp[33];
-    const KmProblem &P = b.p[blockIdx.y];
-    const int bh = blockIdx.x;
+    const KmProblem &P = b.p[blockIdx.z];
+    const int bh = blockIdx.y;
     const int64_t total = (int64_t)P.C * nblk;
-    int32_t *h = P.blockhist + (int64_t)bh * total;
-    int carry = 0;
-    for (int64_t base = 0; base < total; base += blockDim.x) {
-        const int64_t i = base + threadIdx.x;
-        const int v = i < total ? h[i] : 0;
-        int tot;
-        const int ex = block_excl_scan(v, tmp, tot);
-        if (i < total) h[i] = carry + ex;
-        carry += tot;
+    const int64_t t0 = (int64_t)blockIdx.x * kScanTile;
+    if (t0 >= total) return;
+    const int32_t *h = P.blockhist + (int64_t)bh * total;
+    int v = 0;
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+        const int64_t e = t0 + (int64_t)i * kScanThreads + threadIdx.x;
+        v += e < total ? h[e] : 0;
     }
-    __syncthreads();
+    int tot;
+    block_excl_scan(v, tmp, tot);
+    const int ntiles = (int)((total + kScanTile - 1) / kScanTile);
+    if (threadIdx.x == 0) P.tilesum[(int64_t)bh * ntiles + blockIdx.x] = tot;
+}
+
+__global__ void __launch_bounds__(kScanThreads) km_scan_apply_kernel(KmBatch b, int nblk)
+{
+    __shared__ int tmp[33];
+    const KmProblem &P = b.p[blockIdx.z];
+    const int bh = blockIdx.y;
+    const int64_t total = (int64_t)P.C * nblk;
+    const int64_t t0 = (int64_t)blockIdx.x * kScanTile;
+    if (t0 >= total) return;
+    const int ntiles = (int)((total + kScanTile - 1) / kScanTile);
+    const int32_t *ts = P.tilesum + (int64_t)bh * ntiles;
+    int before = 0;
+    for (int i = threadIdx.x; i < (int)blockIdx.x; i += kScanThreads) before += ts[i];
+    int carry;
+    block_excl_scan(before, tmp, carry);  // carry = sum of the tiles before this one
+    int32_t *h = P.blockhist + (int64_t)bh * total;
+    // thread-contiguous counters, so a thread's exclusive prefix is local
+    const int64_t e0 = t0 + (int64_t)threadIdx.x * kScanPer;
+    int v[kScanPer], s = 0;
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+        v[i] = e0 + i < total ? h[e0 + i] : 0;
+        s += v[i];
+    }
+    int tot;
+    int ex = carry + block_excl_scan(s, tmp, tot);
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+        if (e0 + i < total) h[e0 + i] = ex;
+        ex += v[i];
+    }
+}
+
+__global__ void km_starts_kernel(KmBatch b, int N, int nblk)
+{
+    const KmProblem &P = b.p[blockIdx.z];
+    const int bh = blockIdx.y;
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c > P.C) return;
+    const int32_t *h = P.blockhist + (int64_t)bh * P.C * nblk;
     int32_t *start = P.start + (int64_t)bh * (P.C + 1);
-    for (int c = threadIdx.x; c <= P.C; c += blockDim.x) start[c] = c < P.C ? h[(int64_t)c * nblk] : N;
-    __syncthreads();
-    for (int c = threadIdx.x; c < P.C; c += blockDim.x)
-        P.sizes[(int64_t)bh * P.C + c] = start[c + 1] - start[c];
+    const int s0 = c < P.C ? h[(int64_t)c * nblk] : N;
+    start[c] = s0;
+    if (c < P.C) {
+        const int s1 = c + 1 < P.C ? h[(int64_t)(c + 1) * nblk] : N;
+        P.sizes[(int64_t)bh * P.C + c] = s1 - s0;
+    }
 }
 
 // Rows of a block land at base[c][blk] + (rank among earlier rows of label c
@@ -312,7 +387,7 @@ __global__ void __launch_bounds__(1024) km_reduce_kernel(KmBatch b, int N, int D
     const int col = threadIdx.x % colsP, slice = threadIdx.x / colsP;
     const int32_t *start = P.start + (int64_t)bh * (P.C + 1);
     const int st = start[c], sz = start[c + 1] - st;
-    const int S = fixed_shift(P.maxabs, N);
+    const int S = fixed_shift(P.maxabs + bh, N);
     const double scale = ldexp(1.0, S);
     long long acc = 0;
     if (col < dn) {
@@ -377,7 +452,7 @@ __global__ void __launch_bounds__(kSegWarps * 32, 3) km_accum_kernel(KmBatch b, 
     const int32_t *perm = P.perm + (int64_t)bh * N;
     const __nv_bfloat16 *X = P.X + (int64_t)bh * N * D + P.dim_off + d0;
     unsigned long long *sums = P.sums + (int64_t)bh * C * dn + d0;
-    const float scale = ldexpf(1.f, fixed_shift(P.maxabs, N));
+    const float scale = ldexpf(1.f, fixed_shift(P.maxabs + bh, N));
     // the warp's member rows, read once and coalesced
     int32_t *rows = rows_sh[warp];
     for (int t = lane; t < kSegRows; t += 32) rows[t] = p0 + t < p1 ? perm[p0 + t] : 0;
@@ -449,7 +524,7 @@ __global__ void __launch_bounds__(128) km_finalize_kernel(KmBatch b, int N)
     const int dn = P.dim_n;
     const int32_t *start = P.start + (int64_t)bh * (P.C + 1);
     const int sz = start[c + 1] - start[c];
-    const double scale = ldexp(1.0, fixed_shift(P.maxabs, N));
+    const double scale = ldexp(1.0, fixed_shift(P.maxabs + bh, N));
     unsigned long long *sums = P.sums + ((int64_t)bh * P.C + c) * dn;
     float *cent = P.cent + ((int64_t)bh * P.C + c) * dn;
     if (d < dn) {
@@ -505,7 +580,7 @@ void km_fixup_launch(const KmProblem &P, int BH, int N, int D, const int32_t *fi
                      cudaStream_t st)
 {
     (void)BH;
-    km_fixup_kernel<<<148 * 4, 256, 0, st>>>(P, N, D, fix_list, fix_count);
+    km_fixup_kernel<<<148 * 8, kFixWarps * 32, 0, st>>>(P, N, D, fix_list, fix_count);
     count_launches(1);
 }
 
@@ -515,8 +590,11 @@ void launch_km_sort(const KmBatch &b, int BH, int N, cudaStream_t st)
     const size_t smem = (size_t)max_C(b) * sizeof(int);
     km_hist_kernel<<<dim3(nblk, BH, b.count), 32, smem, st>>>(b, N, nblk);
     count_launches(1);
-    km_scan_kernel<<<dim3(BH, b.count), 1024, 0, st>>>(b, N, nblk);
-    count_launches(1);
+    const int ntiles = (int)(((int64_t)max_C(b) * nblk + kScanTile - 1) / kScanTile);
+    km_scan_tiles_kernel<<<dim3(ntiles, BH, b.count), kScanThreads, 0, st>>>(b, nblk);
+    km_scan_apply_kernel<<<dim3(ntiles, BH, b.count), kScanThreads, 0, st>>>(b, nblk);
+    km_starts_kernel<<<dim3((max_C(b) + 256) / 256, BH, b.count), 256, 0, st>>>(b, N, nblk);
+    count_launches(3);
     km_scatter_kernel<<<dim3(nblk, BH, b.count), 32, smem, st>>>(b, N, nblk);
     count_launches(1);
 }

@@ -15,7 +15,7 @@
 // cudaGetSymbolAddress (with that device current) and caches it; make that
 // first call before any stream capture.  All calls share the array and it
 // keeps the last call's contents: the one region that must start at zero (the
-// max-|x| word) is cleared at the start of every call, everything else is
+// per-head max-|x| words) is cleared at the start of every call, everything else is
 // fully rewritten.  Calls whose device work overlaps (e.g. on two streams)
 // race on the array and must be serialised by the caller.
 #include <mutex>
@@ -44,17 +44,18 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {nullptr};
 
-// Max |x| of the rows' columns (the fixed-point scale of the centroid sums).
-__global__ void maxabs_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows, int D, int dim_off, int dim_n,
-                              uint32_t *out)
+// Max |x| over every column of the rows (the fixed-point scale of the
+// centroid sums).  scope_plan takes the same maximum over the whole rotated
+// key (or query) rows for every subspace, so the two scales, and hence the
+// rounding of the centroid sums, agree when x is the plan's rotated tensor.
+// One maximum per (batch, head) (grid y), like the plan's.
+__global__ void maxabs_kernel(const __nv_bfloat16 *__restrict__ x, int64_t n, uint32_t *out)
 {
     float m = 0.f;
-    const int64_t total = rows * dim_n;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / dim_n;
-        const int k = (int)(i % dim_n);
-        m = fmaxf(m, fabsf(__bfloat162float(x[r * D + dim_off + k])));
-    }
+    const __nv_bfloat16 *xb = x + (int64_t)blockIdx.y * n;
+    out += blockIdx.y;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        m = fmaxf(m, fabsf(__bfloat162float(xb[i])));
     m = warp_max(m);
     if ((threadIdx.x & 31) == 0) atomicMax(out, __float_as_uint(m));
 }
@@ -67,7 +68,9 @@ extern "C" size_t scope_kmeans_noalloc_scratch_bytes(int64_t B, int64_t H, int64
 {
     if (B < 1 || H < 1 || N < 1 || C < 1) return 0;
     const int64_t BH = B * H, nblk = (N + kSortBlk - 1) / kSortBlk;
-    return align256(64) + align256((size_t)BH * N * 4) + align256((size_t)BH * C * nblk * 4) +
+    const int64_t tiles = ((int64_t)C * nblk + kScanTileCounters - 1) / kScanTileCounters;
+    return align256((size_t)BH * 4) + align256((size_t)BH * N * 4) + align256((size_t)BH * C * nblk * 4) +
+           align256((size_t)BH * tiles * 4) +
            align256((size_t)BH * (C + 1) * 4) + 2 * align256((size_t)BH * C * 4);
 }
 
@@ -77,9 +80,19 @@ extern "C" scope_status scope_kmeans_noalloc(const scope_tensor *x, int32_t dim_
 {
     if (!x || !x->ptr || !labels || !centroids) return scope_set_error(SCOPE_EINVAL, "noalloc: null pointer");
     if (((uintptr_t)x->ptr) & 15) return scope_set_error(SCOPE_EALIGN, "noalloc: x not 16-byte aligned");
+    if ((((uintptr_t)labels) | ((uintptr_t)centroids)) & 3)
+        return scope_set_error(SCOPE_EALIGN, "noalloc: labels and centroids must be 4-byte aligned");
     if (x->dtype != SCOPE_BF16) return scope_set_error(SCOPE_EDTYPE, "noalloc: x must be bf16");
     if (x->B < 1 || x->H < 1 || x->N < 1 || (x->D != 64 && x->D != 128))
         return scope_set_error(SCOPE_ESHAPE, "noalloc: x must be [B,H,N,D] with D in {64, 128}");
+    {
+        const int64_t *sd = x->strides;
+        const bool zero = sd[0] == 0 && sd[1] == 0 && sd[2] == 0 && sd[3] == 0;
+        const bool dense = sd[3] == 1 && sd[2] == x->D && sd[1] == x->N * x->D && (x->B == 1 || sd[0] == x->H * x->N * x->D);
+        if (!zero && !dense) return scope_set_error(SCOPE_ESHAPE, "noalloc: x must be contiguous");
+    }
+    if (x->B * x->H > 65535 || x->B * x->H * x->N >= ((int64_t)1 << 31))
+        return scope_set_error(SCOPE_ESHAPE, "noalloc: need B*H <= 65535 and B*H*N < 2^31");
     if (dim_off < 0 || dim_n < 1 || dim_off + dim_n > x->D)
         return scope_set_error(SCOPE_ESHAPE, "noalloc: column range outside [0, D)");
     if (C < 1 || C > kMaxClusters || C > x->N)
@@ -97,6 +110,13 @@ extern "C" scope_status scope_kmeans_noalloc(const scope_tensor *x, int32_t dim_
     int major = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     if (major != 10) return scope_set_error(SCOPE_EDEVICE, "noalloc: libscope.so is built for sm_100a");
+    {
+        // the scratch address below is the current device's: the stream's
+        // kernels must run there too
+        int sdev = -1;
+        if (cudaStreamGetDevice((cudaStream_t)stream, &sdev) != cudaSuccess || sdev != dev)
+            return scope_set_error(SCOPE_EDEVICE, "noalloc: the stream belongs to another device than the current one");
+    }
     char *base;
     {
         std::lock_guard<std::mutex> lock(g_mu);
@@ -118,7 +138,7 @@ extern "C" scope_status scope_kmeans_noalloc(const scope_tensor *x, int32_t dim_
         cur += align256(bytes);
         return p;
     };
-    uint32_t *stats = (uint32_t *)take(64);
+    uint32_t *stats = (uint32_t *)take((size_t)BH * 4);
     KmProblem P{};
     P.X = (const __nv_bfloat16 *)x->ptr;
     P.maxabs = stats;
@@ -129,6 +149,7 @@ extern "C" scope_status scope_kmeans_noalloc(const scope_tensor *x, int32_t dim_
     P.cent = centroids;
     P.perm = (int32_t *)take((size_t)BH * N * 4);
     P.blockhist = (int32_t *)take((size_t)BH * C * nblk * 4);
+    P.tilesum = (int32_t *)take((size_t)BH * (((int64_t)C * nblk + kScanTileCounters - 1) / kScanTileCounters) * 4);
     P.start = (int32_t *)take((size_t)BH * (C + 1) * 4);
     P.sizes = (int32_t *)take((size_t)BH * C * 4);
     P.cn = (float *)take((size_t)BH * C * 4);
@@ -136,8 +157,8 @@ extern "C" scope_status scope_kmeans_noalloc(const scope_tensor *x, int32_t dim_
     b.p[0] = P;
     b.count = 1;
 
-    cudaMemsetAsync(stats, 0, 64, s);
-    maxabs_kernel<<<592, 256, 0, s>>>(P.X, BH * N, (int)x->D, dim_off, dim_n, stats);
+    cudaMemsetAsync(stats, 0, (size_t)BH * 4, s);
+    maxabs_kernel<<<dim3((unsigned)((4 * 148 + BH - 1) / BH), (unsigned)BH), 256, 0, s>>>(P.X, N * x->D, stats);
     count_launches(1);
     launch_km_init(b, (int)BH, (int)N, (int)x->D, init_seed, s);
     for (int it = 0; it < iters; ++it) {

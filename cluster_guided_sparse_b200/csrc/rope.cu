@@ -8,9 +8,10 @@
 //
 // HBM-bound: one 16-byte bf16 vector of output per thread, inputs read with
 // 16/32-byte vector loads, (cos, sin) from a small per-axis fp64 table that
-// stays in L1.  The same pass emits ||x||^2 of every stored (rounded) row and the
-// tensor's max |x|, which later stages use for the assignment error bound
-// and the fixed-point scale of the centroid sums.
+// stays in L1.  The same pass emits ||x||^2 of every stored (rounded) row and
+// the max |x| of every (batch, head), which later stages use for the
+// assignment error bound and the fixed-point scale of the centroid sums (per
+// head, so a head's results never depend on the other heads of the call).
 #include "common.cuh"
 
 namespace scope {
@@ -63,7 +64,7 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, flo
 // One thread = 8 consecutive dims of one row; D/8 threads per row (8 or 16).
 template <typename TIn>
 __global__ void __launch_bounds__(256) rope_apply_kernel(
-    const TIn *__restrict__ in, __nv_bfloat16 *__restrict__ out, float *__restrict__ norm2,
+    const TIn *__restrict__ in, RowStrides rs, __nv_bfloat16 *__restrict__ out, float *__restrict__ norm2,
     uint32_t *__restrict__ maxabs, const double2 *__restrict__ tab, int64_t rows, int N, int D,
     int Hh, int W, int dt, int dh, int maxL, int maxP, int use_rope)
 {
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(
     float ss = 0.f, mx = 0.f;
     if (valid) {
         float x[8];
-        load8<TIn>(in + row * D + c8 * 8, x);
+        load8<TIn>(in + rs.row(row / N, row % N) + c8 * 8, x);
         // The rotation runs in double and is rounded once to bf16, so every
         // stored element is the correctly rounded rotation of its input (in
         // fp32 a near-zero result of x0*c - x1*s can be off by more than one
@@ -116,14 +117,21 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(
     // Row norm over the tpr lanes that share the row (tpr divides 32).
     for (int o = tpr >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (norm2 && valid && c8 == 0) norm2[row] = ss;
-    // max |x| of the block, then one atomic (per-warp atomics on one word
-    // would serialise)
-    mx = warp_max(mx);
-    if ((threadIdx.x & 31) == 0) bmax[threadIdx.x >> 5] = mx;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, bmax[w]);
-        atomicMax(maxabs, __float_as_uint(mx));
+    // max |x| per (batch, head): the block's rows nearly always belong to one
+    // head, whose maximum then takes one atomic (per-warp atomics on one word
+    // would serialise); a block that straddles two heads updates per thread.
+    const int64_t first = ((int64_t)blockIdx.x * blockDim.x) >> sh;
+    const int64_t last = min(rows - 1, first + (int64_t)(blockDim.x >> sh) - 1);
+    if (first / N == last / N) {
+        mx = warp_max(mx);
+        if ((threadIdx.x & 31) == 0) bmax[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            for (int w = 1; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, bmax[w]);
+            atomicMax(maxabs + first / N, __float_as_uint(mx));
+        }
+    } else if (valid && mx > 0.f) {
+        atomicMax(maxabs + row / N, __float_as_uint(mx));
     }
 }
 
@@ -135,7 +143,8 @@ void launch_rope_table(double2 *tab, int T, int Hh, int W, int dt, int dh, int d
     count_launches(1);
 }
 
-void launch_rope_apply(const void *in, bool in_f32, __nv_bfloat16 *out, float *norm2, uint32_t *maxabs,
+void launch_rope_apply(const void *in, const RowStrides &rs, bool in_f32, __nv_bfloat16 *out, float *norm2,
+                       uint32_t *maxabs,
                        const double2 *tab, int64_t rows, int N, int D, int Hh, int W, int dt, int dh,
                        int maxL, int maxP, int use_rope, cudaStream_t st)
 {
@@ -143,20 +152,24 @@ void launch_rope_apply(const void *in, bool in_f32, __nv_bfloat16 *out, float *n
     const int64_t blocks = (threads + 255) / 256;
     if (in_f32)
         rope_apply_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
-            (const float *)in, out, norm2, maxabs, tab, rows, N, D, Hh, W, dt, dh, maxL, maxP, use_rope);
+            (const float *)in, rs, out, norm2, maxabs, tab, rows, N, D, Hh, W, dt, dh, maxL, maxP, use_rope);
     else
         rope_apply_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)in, out, norm2, maxabs, tab, rows, N, D, Hh, W, dt, dh, maxL, maxP,
+            (const __nv_bfloat16 *)in, rs, out, norm2, maxabs, tab, rows, N, D, Hh, W, dt, dh, maxL, maxP,
             use_rope);
     count_launches(1);
 }
 
-// bf16 copy of an f32 tensor (V of f32 calls; the tensor-core path reads bf16).
-__global__ void to_bf16_kernel(const float4 *__restrict__ in, uint2 *__restrict__ out, int64_t n4)
+// Contiguous bf16 copy of a (possibly strided) f32 tensor (V of f32 calls; the
+// tensor-core path reads bf16).  One thread = 4 elements of one row.
+__global__ void to_bf16_kernel(const float *__restrict__ in, RowStrides rs, uint2 *__restrict__ out, int64_t n4,
+                               int N, int D)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n4) return;
-    const float4 f = in[i];
+    const int64_t row = i / (D / 4);
+    const int c4 = (int)(i % (D / 4));
+    const float4 f = *reinterpret_cast<const float4 *>(in + rs.row(row / N, row % N) + 4 * c4);
     __nv_bfloat162 a = __floats2bfloat162_rn(f.x, f.y), b = __floats2bfloat162_rn(f.z, f.w);
     uint2 u;
     u.x = *reinterpret_cast<uint32_t *>(&a);
@@ -164,10 +177,11 @@ __global__ void to_bf16_kernel(const float4 *__restrict__ in, uint2 *__restrict_
     out[i] = u;
 }
 
-void launch_to_bf16(const float *in, __nv_bfloat16 *out, int64_t n, cudaStream_t st)
+void launch_to_bf16(const float *in, const RowStrides &rs, __nv_bfloat16 *out, int64_t n, int N, int D,
+                    cudaStream_t st)
 {
     const int64_t n4 = n / 4;
-    to_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>((const float4 *)in, (uint2 *)out, n4);
+    to_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(in, rs, (uint2 *)out, n4, N, D);
     count_launches(1);
 }
 

@@ -15,9 +15,9 @@
 namespace scope {
 // kernels.cu launchers
 void launch_rope_table(double2 *, int, int, int, int, int, int, double, int, int, cudaStream_t);
-void launch_rope_apply(const void *, bool, __nv_bfloat16 *, float *, uint32_t *, const double2 *, int64_t, int, int,
-                       int, int, int, int, int, int, int, cudaStream_t);
-void launch_to_bf16(const float *, __nv_bfloat16 *, int64_t, cudaStream_t);
+void launch_rope_apply(const void *, const RowStrides &, bool, __nv_bfloat16 *, float *, uint32_t *, const double2 *,
+                       int64_t, int, int, int, int, int, int, int, int, int, cudaStream_t);
+void launch_to_bf16(const float *, const RowStrides &, __nv_bfloat16 *, int64_t, int, int, cudaStream_t);
 cudaError_t km_configure();
 void launch_km_init(const KmBatch &, int, int, int, uint32_t, cudaStream_t);
 void launch_km_assign_direct(const KmBatch &, int, int, int, cudaStream_t);
@@ -38,18 +38,21 @@ void launch_items(const int32_t *, int32_t *, int32_t *, int32_t *, int32_t *, u
 cudaError_t select_configure();
 cudaError_t attn_tc_configure();
 int attn_tc_max_items(int BH, int N, int Cq);
-bool launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, __nv_bfloat16 *, int4 *,
-                    int32_t *, int, const int32_t *, const int32_t *, const int32_t *, const long long *,
-                    const int32_t *, const int32_t *, int32_t *, float *, int, int, int, int, cudaStream_t);
-void launch_compensate(const __nv_bfloat16 *, const __nv_bfloat16 *, const int32_t *, const int32_t *, const int32_t *,
-                       const int32_t *, const int32_t *, const int32_t *, const float *, float *, const long long *,
-                       const int32_t *, const int32_t *, const float *, __nv_bfloat16 *, int, int, int, int, int,
-                       cudaStream_t);
+bool launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, const RowStrides &,
+                    __nv_bfloat16 *, const RowStrides &, int4 *, int32_t *, int, const int32_t *, const int32_t *,
+                    const int32_t *, const long long *, const int32_t *, const int32_t *, int32_t *, float *, int, int,
+                    int, int, cudaStream_t);
+void launch_compensate(const __nv_bfloat16 *, const __nv_bfloat16 *, const RowStrides &, const int32_t *,
+                       const int32_t *, const int32_t *, const int32_t *, const int32_t *, const int32_t *,
+                       const float *, float *, const long long *, const int32_t *, const int32_t *, const float *,
+                       __nv_bfloat16 *, const RowStrides &, int, int, int, int, int, cudaStream_t);
+void launch_wait_timeout(int32_t *err, long long limit, cudaStream_t st);
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
                    const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch, int Cw,
                    int BH, float top_p,
                    float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes, int32_t *r, int32_t *n,
-                   int32_t *kh, long long *offsets, int32_t *indices, int online, cudaStream_t st);
+                   int32_t *kh, long long *offsets, int32_t *indices, int online, void *state, cudaStream_t st);
+size_t selection_state_bytes(int64_t clusters);
 }  // namespace scope
 
 using namespace scope;
@@ -85,13 +88,16 @@ struct Layout {
     int Cq, C[3], ds[3], off[3], Csum, P, Pcap, nblk, max_work, maxL, maxP;
     bool f32, bisect;
     int64_t cap;
-    size_t qr, kr, qnorm, tab, stats, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist;
-    size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3];
-    size_t lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
+    size_t qr, kr, qnorm, tab, stats, maxabs, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist, q_tsum;
+    size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3], k_tsum[3];
+    size_t sel_state, lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
     size_t bis_order, bis_delta, bis_aux, q_chi, q_clo, q_sums, k_sums[3], sums_bytes, lse, vmean;
     bool comp;
     size_t total;
 };
+
+// Tiles of the parallel scan over a problem's C x nblk block counters.
+int64_t scan_tiles(int64_t C, int64_t nblk) { return (C * nblk + kScanTileCounters - 1) / kScanTileCounters; }
 
 size_t take(size_t &cur, size_t bytes)
 {
@@ -123,8 +129,8 @@ bool tensor_ok(const scope_tensor *t, const char *name, scope_status *st)
         *st = fail(SCOPE_ESHAPE, "%s: head dim must be 64 or 128 (got %lld)", name, (long long)t->D);
         return false;
     }
-    if (t->B * t->H * t->N >= (int64_t)1 << 31) {
-        *st = fail(SCOPE_ESHAPE, "%s: B*H*N must be < 2^31", name);
+    if (t->B * t->H * t->N >= (int64_t)1 << 31 || t->B * t->H > 65535) {
+        *st = fail(SCOPE_ESHAPE, "%s: B*H*N must be < 2^31 and B*H <= 65535", name);
         return false;
     }
     if (t->N > (1 << 24)) {
@@ -135,7 +141,71 @@ bool tensor_ok(const scope_tensor *t, const char *name, scope_status *st)
         *st = fail(SCOPE_EDTYPE, "%s: dtype must be f32 or bf16", name);
         return false;
     }
+    const int64_t *sd = t->strides;
+    if (sd[0] == 0 && sd[1] == 0 && sd[2] == 0 && sd[3] == 0) return true;  // contiguous
+    const int64_t elt = t->dtype == SCOPE_F32 ? 4 : 2;
+    if (sd[3] != 1 || sd[0] < 0 || sd[1] < 0 || sd[2] < 0) {
+        *st = fail(SCOPE_ESHAPE, "%s: strides[3] must be 1 and the others >= 0", name);
+        return false;
+    }
+    for (int i = 0; i < 3; ++i)
+        if ((sd[i] * elt) % 16) {
+            *st = fail(SCOPE_ESHAPE, "%s: strides[%d] * element size must be a multiple of 16 bytes", name, i);
+            return false;
+        }
+    // distinct (b, h, n) must not share a row: with the dimensions of extent
+    // > 1 sorted by stride, each stride must reach past the previous
+    // dimension's whole extent (the row itself is D elements wide)
+    int64_t st_[4] = {1, sd[2], sd[1], sd[0]}, ex[4] = {t->D, t->N, t->H, t->B};
+    int m = 0;
+    for (int i = 0; i < 4; ++i)
+        if (ex[i] > 1 || i == 0) {
+            if (st_[i] == 0) {
+                *st = fail(SCOPE_ESHAPE, "%s: strides make distinct rows overlap", name);
+                return false;
+            }
+            st_[m] = st_[i];
+            ex[m] = ex[i];
+            ++m;
+        }
+    for (int i = 1; i < m; ++i)
+        for (int j = i; j > 0 && st_[j] < st_[j - 1]; --j) {
+            int64_t a = st_[j]; st_[j] = st_[j - 1]; st_[j - 1] = a;
+            a = ex[j]; ex[j] = ex[j - 1]; ex[j - 1] = a;
+        }
+    for (int i = 1; i < m; ++i)
+        if (st_[i] < st_[i - 1] * ex[i - 1]) {
+            *st = fail(SCOPE_ESHAPE, "%s: strides make distinct rows overlap", name);
+            return false;
+        }
     return true;
+}
+
+// Row addressing of a caller tensor (all-zero strides: contiguous).
+RowStrides rows_of(const scope_tensor *t)
+{
+    RowStrides r;
+    r.H = (int)t->H;
+    if (t->strides[0] == 0 && t->strides[1] == 0 && t->strides[2] == 0 && t->strides[3] == 0) {
+        r.sN = t->D;
+        r.sH = t->N * t->D;
+        r.sB = t->H * t->N * t->D;
+    } else {
+        r.sB = t->strides[0];
+        r.sH = t->strides[1];
+        r.sN = t->strides[2];
+    }
+    return r;
+}
+
+RowStrides contiguous_rows(int64_t H, int64_t N, int64_t D)
+{
+    RowStrides r;
+    r.H = (int)H;
+    r.sN = D;
+    r.sH = N * D;
+    r.sB = H * N * D;
+    return r;
 }
 
 bool same_shape(const scope_tensor *a, const scope_tensor *b)
@@ -229,6 +299,7 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.qnorm = take(cur, BH * N * 4);
     L.tab = take(cur, (size_t)3 * L.maxL * L.maxP * 16);
     L.stats = take(cur, 64);
+    L.maxabs = take(cur, 2 * BH * 4);
     L.q_lab = take(cur, BH * N * 4);
     L.q_cent = take(cur, BH * L.Cq * D * 4);
     L.q_cn = take(cur, BH * L.Cq * 4);
@@ -236,6 +307,7 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.q_perm = take(cur, BH * N * 4);
     L.q_start = take(cur, BH * (L.Cq + 1) * 4);
     L.q_bhist = take(cur, BH * L.Cq * L.nblk * 4);
+    L.q_tsum = take(cur, BH * scan_tiles(L.Cq, L.nblk) * 4);
     L.fix = take(cur, BH * N * 4 + 16);
     L.q_chi = take(cur, BH * L.Cq * D * 2);
     L.q_clo = take(cur, BH * L.Cq * D * 2);
@@ -260,8 +332,10 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
         L.k_perm[s] = take(cur, BH * N * 4);
         L.k_start[s] = take(cur, BH * (L.C[s] + 1) * 4);
         L.k_bhist[s] = take(cur, BH * L.C[s] * L.nblk * 4);
+        L.k_tsum[s] = take(cur, BH * scan_tiles(L.C[s], L.nblk) * 4);
     }
     L.lut = take(cur, BH * L.Cq * L.Csum * 4);
+    L.sel_state = take(cur, selection_state_bytes(BH * L.Cq));
     L.item_hist = take(cur, BH * L.P * 4);
     L.item_id = take(cur, BH * L.Pcap * 4);
     L.item_cnt = take(cur, BH * L.Pcap * 4);
@@ -336,15 +410,17 @@ static void rope_both(const Layout &L, char *ws, const scope_tensor *q, const sc
 {
     const bool rope = g && g->T > 0;
     uint32_t *stats = at<uint32_t>(ws, L.stats);
+    uint32_t *maxabs = at<uint32_t>(ws, L.maxabs);
     cudaMemsetAsync(stats, 0, 64, st);
+    cudaMemsetAsync(maxabs, 0, 2 * L.BH * 4, st);
     if (rope)
         launch_rope_table(at<double2>(ws, L.tab), g->T, g->Hh, g->W, p->d_t, p->d_h, p->d_w, p->theta, L.maxL, L.maxP,
                           st);
     const int Hh = rope ? g->Hh : 1, W = rope ? g->W : 1;
-    launch_rope_apply(q->ptr, L.f32, at<__nv_bfloat16>(ws, L.qr), at<float>(ws, L.qnorm), stats + 0,
+    launch_rope_apply(q->ptr, rows_of(q), L.f32, at<__nv_bfloat16>(ws, L.qr), at<float>(ws, L.qnorm), maxabs,
                       at<double2>(ws, L.tab), L.BH * L.N, (int)L.N, (int)L.D, Hh, W, p->d_t, p->d_h, L.maxL, L.maxP,
                       rope ? 1 : 0, st);
-    launch_rope_apply(k->ptr, L.f32, at<__nv_bfloat16>(ws, L.kr), nullptr, stats + 1, at<double2>(ws, L.tab),
+    launch_rope_apply(k->ptr, rows_of(k), L.f32, at<__nv_bfloat16>(ws, L.kr), nullptr, maxabs + L.BH, at<double2>(ws, L.tab),
                       L.BH * L.N, (int)L.N, (int)L.D, Hh, W, p->d_t, p->d_h, L.maxL, L.maxP, rope ? 1 : 0, st);
 }
 
@@ -352,7 +428,7 @@ static KmProblem key_problem(const Layout &L, char *ws, int s)
 {
     KmProblem P{};
     P.X = at<__nv_bfloat16>(ws, L.kr);
-    P.maxabs = at<uint32_t>(ws, L.stats) + 1;
+    P.maxabs = at<uint32_t>(ws, L.maxabs) + L.BH;
     P.dim_off = L.off[s];
     P.dim_n = L.ds[s];
     P.C = L.C[s];
@@ -363,6 +439,7 @@ static KmProblem key_problem(const Layout &L, char *ws, int s)
     P.perm = at<int32_t>(ws, L.k_perm[s]);
     P.start = at<int32_t>(ws, L.k_start[s]);
     P.blockhist = at<int32_t>(ws, L.k_bhist[s]);
+    P.tilesum = at<int32_t>(ws, L.k_tsum[s]);
     P.sums = at<unsigned long long>(ws, L.k_sums[s]);
     return P;
 }
@@ -371,7 +448,7 @@ static KmProblem query_problem(const Layout &L, char *ws)
 {
     KmProblem P{};
     P.X = at<__nv_bfloat16>(ws, L.qr);
-    P.maxabs = at<uint32_t>(ws, L.stats);
+    P.maxabs = at<uint32_t>(ws, L.maxabs);
     P.dim_off = 0;
     P.dim_n = (int)L.D;
     P.C = L.Cq;
@@ -382,6 +459,7 @@ static KmProblem query_problem(const Layout &L, char *ws)
     P.perm = at<int32_t>(ws, L.q_perm);
     P.start = at<int32_t>(ws, L.q_start);
     P.blockhist = at<int32_t>(ws, L.q_bhist);
+    P.tilesum = at<int32_t>(ws, L.q_tsum);
     P.sums = at<unsigned long long>(ws, L.q_sums);
     return P;
 }
@@ -475,7 +553,7 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
                   L.Cq, L.C[0], L.C[1], L.C[2], BH, p->top_p, 1.0f / sqrtf((float)D), p->k_min,
                   at<int32_t>(ws, L.stats) + 4,
                   at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.r), at<int32_t>(ws, L.n), at<int32_t>(ws, L.kh),
-                  at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, s);
+                  at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, ws + L.sel_state, s);
     if ((st = launch_status("selection")) != SCOPE_OK) return st;
 
     scope_plan_s *h = (scope_plan_s *)malloc(sizeof(scope_plan_s));
@@ -501,11 +579,17 @@ static scope_status check_vo(const scope_tensor *q, const scope_tensor *v, const
     return SCOPE_OK;
 }
 
-static const __nv_bfloat16 *v_bf16(const Layout &L, char *ws, const scope_tensor *v, cudaStream_t s)
+// bf16 V for the attention: the caller's rows, or a contiguous bf16 copy of
+// f32 ones in the workspace (`vs` receives the row addressing of either).
+static const __nv_bfloat16 *v_bf16(const Layout &L, char *ws, const scope_tensor *v, RowStrides *vs, cudaStream_t s)
 {
-    if (v->dtype == SCOPE_BF16) return (const __nv_bfloat16 *)v->ptr;
+    if (v->dtype == SCOPE_BF16) {
+        *vs = rows_of(v);
+        return (const __nv_bfloat16 *)v->ptr;
+    }
     __nv_bfloat16 *vb = at<__nv_bfloat16>(ws, L.vb);
-    launch_to_bf16((const float *)v->ptr, vb, L.BH * L.N * L.D, s);
+    launch_to_bf16((const float *)v->ptr, rows_of(v), vb, L.BH * L.N * L.D, (int)L.N, (int)L.D, s);
+    *vs = contiguous_rows(L.H, L.N, L.D);
     return vb;
 }
 
@@ -525,8 +609,10 @@ extern "C" scope_status scope_attn(const scope_tensor *q, const scope_tensor *k,
     cudaStream_t s = (cudaStream_t)stream;
     if ((st = check_device(s)) != SCOPE_OK) return st;
     char *ws = plan->ws;
-    const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
-    if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
+    RowStrides vs;
+    const __nv_bfloat16 *vb = v_bf16(L, ws, v, &vs, s);
+    const RowStrides os = rows_of(o);
+    if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, vs, (__nv_bfloat16 *)o->ptr, os,
                    at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, at<int32_t>(ws, L.q_sizes),
                    at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start), at<long long>(ws, L.offsets),
                    at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n), at<int32_t>(ws, L.stats) + 4,
@@ -534,11 +620,11 @@ extern "C" scope_status scope_attn(const scope_tensor *q, const scope_tensor *k,
         return fail(SCOPE_ECUDA, "scope_attn: tensor map encoding failed");
     if (L.comp)
         // ClusterAttention: excluded key clusters enter through their mean key and value
-        launch_compensate(at<__nv_bfloat16>(ws, L.qr), vb, at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start),
+        launch_compensate(at<__nv_bfloat16>(ws, L.qr), vb, vs, at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start),
                           at<int32_t>(ws, L.k_perm[0]), at<int32_t>(ws, L.k_start[0]), at<int32_t>(ws, L.k_codes),
                           at<int32_t>(ws, L.k_sizes[0]), at<float>(ws, L.k_cent[0]), at<float>(ws, L.vmean),
                           at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n),
-                          at<float>(ws, L.lse), (__nv_bfloat16 *)o->ptr, (int)L.BH, (int)L.N, (int)L.D, L.Cq,
+                          at<float>(ws, L.lse), (__nv_bfloat16 *)o->ptr, os, (int)L.BH, (int)L.N, (int)L.D, L.Cq,
                           L.C[0], s);
     return launch_status("scope_attn");
 }
@@ -562,6 +648,7 @@ static Layout dense_layout(const scope_tensor *q, const scope_grid *g, const sco
     L.qnorm = take(cur, L.BH * L.N * 4);
     L.tab = take(cur, (size_t)3 * L.maxL * L.maxP * 16);
     L.stats = take(cur, 64);
+    L.maxabs = take(cur, 2 * L.BH * 4);
     L.vb = take(cur, L.f32 ? L.BH * L.N * L.D * 2 : 0);
     L.max_work = attn_tc_max_items((int)L.BH, (int)L.N, 0);
     L.work = take(cur, (size_t)L.max_work * 16);
@@ -611,9 +698,10 @@ extern "C" scope_status scope_dense_attn(const scope_tensor *q, const scope_tens
     if ((st = check_device(s)) != SCOPE_OK) return st;
     char *ws = (char *)workspace;
     rope_both(L, ws, q, k, has_grid ? grid : nullptr, p, s);
-    const __nv_bfloat16 *vb = v_bf16(L, ws, v, s);
-    if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, (__nv_bfloat16 *)o->ptr,
-                        at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, nullptr, nullptr, nullptr,
+    RowStrides vs;
+    const __nv_bfloat16 *vb = v_bf16(L, ws, v, &vs, s);
+    if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, vs, (__nv_bfloat16 *)o->ptr,
+                        rows_of(o), at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, nullptr, nullptr, nullptr,
                         nullptr, nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, nullptr, (int)L.BH, (int)L.N,
                         (int)L.D, 1, s))
         return fail(SCOPE_ECUDA, "scope_dense_attn: tensor map encoding failed");
@@ -670,6 +758,17 @@ extern "C" scope_status scope_sync_status(const scope_plan_t *plan, void *stream
     if (err[0] & kErrTimeout) return fail(SCOPE_ETIMEOUT, "a bounded device wait gave up (detail 0x%x)", err[1]);
     if (err[0]) return fail(SCOPE_EDEVICE, "device range check fired (flags 0x%x, detail 0x%x)", err[0], err[1]);
     return SCOPE_OK;
+}
+
+extern "C" scope_status scope_selftest_wait_timeout(const scope_plan_t *plan, int64_t wait_cycles, void *stream)
+{
+    if (!plan) return fail(SCOPE_EINVAL, "plan: null");
+    if (wait_cycles < 1000 || wait_cycles > 4000000000ll)
+        return fail(SCOPE_EINVAL, "wait_cycles must be in [1e3, 4e9]");
+    scope_status st;
+    if ((st = check_device((cudaStream_t)stream)) != SCOPE_OK) return st;
+    launch_wait_timeout((int32_t *)(plan->ws + plan->L.stats + 16), (long long)wait_cycles, (cudaStream_t)stream);
+    return launch_status("scope_selftest_wait_timeout");
 }
 
 extern "C" void scope_plan_destroy(scope_plan_t *plan) { free(plan); }

@@ -113,17 +113,35 @@ __global__ void key_item_kernel(const int32_t *codes, const int32_t *rank, uint1
     key_item[i] = (uint16_t)rank[(int64_t)bh * P + id];
 }
 
-// -------------------------------------------------------------- radix select
-// Candidates are keys whose 32-bit order key matches `prefix` above the bits
-// still open.  Invariant: above_met < target <= above_met + (candidates'
-// metric), where above_* sum the keys strictly above the candidate range.
+// -------------------------------------------------------------- Top-p select
+// The order of a cluster's keys is (score desc, index asc); a key's place in
+// it depends only on its item's 32-bit order key u = ordered_key(score).
+//
+// The select runs in two stages.  Coarse: every item goes to one of kBuckets
+// buckets by a monotone map of its score onto [smin, smax] of the cluster
+// (so the buckets spread over the scores actually present, instead of
+// crowding into the few exponent bits they share), carrying key counts and
+// softmax masses; the bucket where the running metric from the top reaches
+// the target is found by a scan.  Refine: a radix select on the exact order
+// key (11/11/10 bits) among that bucket's items alone.  Masses are 64-bit
+// fixed point (2^40 units), so every sum is exact and order-free.
+//
+// Items' order keys are computed once per kernel and kept in shared memory
+// when the head has at most kItemCache distinct items (720p: <= 16 384).
+// The Top-p kernel stores, per cluster, the score range, the coarse count
+// histogram and its cut, so the list emission can skip the coarse pass and,
+// when a cluster's final count equals its Top-p count, the whole select.
+constexpr int kBuckets = 2048;
+constexpr int kItemCache = 16384;
+
 struct SelShared {
-    unsigned long long met[2048];
-    int cnt[2048];
+    unsigned long long met[kBuckets];
+    int cnt[kBuckets];
     unsigned long long utmp[33];
     int itmp[33];
-    float fred[32];
+    float fmin[32], fmax[32];
     uint32_t prefix;
+    int coarse;  // the coarse bucket being refined (-1: none)
     unsigned long long above_met, run_met, bucket_met, new_above_met;
     int above_cnt, run_cnt, bucket_cnt, new_above_cnt, bucket;
 };
@@ -134,42 +152,67 @@ __device__ __forceinline__ float item_score(const float *L, int id, int Ch, int 
     return (L[a_t] + L[Ct + a_h]) + L[Ct + Ch + a_w];
 }
 
+__device__ __forceinline__ float key_score(uint32_t u)
+{
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
 __device__ __forceinline__ unsigned long long item_mass(float s, float smax, float inv_sqrt_d)
 {
     const float w = expf((s - smax) * inv_sqrt_d);
     return (unsigned long long)__double2ll_rn((double)w * kMassScale);
 }
 
-// One pass over `width` more bits below `shift + width`; returns false if no
-// bucket satisfied the invariant (cannot happen with exact integer metrics).
-__device__ bool radix_pass(SelShared &S, const float *L, const int32_t *ids, const int32_t *cnts, int n_items,
-                           const SelArgs &a, float smax, bool by_mass, unsigned long long target, int shift,
-                           int width)
-{
-    const int nb = 1 << width;
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-        S.met[i] = 0ull;
-        S.cnt[i] = 0;
+// Monotone (non-decreasing) map of a score onto the coarse buckets; the same
+// fp32 operations in every kernel, so every kernel places an item alike.
+struct CoarseMap {
+    float smin, scale;
+    __device__ __forceinline__ CoarseMap(float lo, float hi)
+    {
+        smin = lo;
+        const float sc = hi > lo ? __fdiv_rn((float)kBuckets, __fsub_rn(hi, lo)) : 0.f;
+        scale = isfinite(sc) ? sc : 0.f;
     }
+    __device__ __forceinline__ int operator()(float s) const
+    {
+        const float t = __fmul_rn(__fsub_rn(s, smin), scale);
+        return t < (float)(kBuckets - 1) ? (int)t : kBuckets - 1;
+    }
+};
+
+// Per cluster, written by the Top-p kernel for the list emission.
+struct ClusterCut {
+    float smin, smax;
+    uint32_t key;     // order key of the last key the Top-p prefix takes
+    int32_t need;     // keys it takes at that key
+    int32_t taken;    // the Top-p count |P_c|
+    int32_t pad[3];
+};
+
+// The order key of item i (cached, or recomputed from the table row).
+struct ItemKeys {
+    const uint32_t *cache;  // null when not cached
+    const float *L;
+    const int32_t *ids;
+    int Ct, Ch, Cw;
+    __device__ __forceinline__ uint32_t operator()(int i) const
+    {
+        return cache ? cache[i] : ordered_key(item_score(L, ids[i], Ch, Cw, Ct));
+    }
+};
+
+// Scans the histogram S.met / S.cnt (nb buckets) from the top bucket down
+// for the bucket where the running metric first reaches `target`, on top of
+// S.above_met / S.above_cnt.  Sets S.bucket (-1 if none), S.bucket_met,
+// S.bucket_cnt and moves S.above_* to the keys strictly above that bucket.
+__device__ void pick_bucket(SelShared &S, int nb, unsigned long long target)
+{
     if (threadIdx.x == 0) {
         S.run_met = 0ull;
         S.run_cnt = 0;
         S.bucket = -1;
     }
     __syncthreads();
-    const uint32_t pre = S.prefix;
-    const int hi = shift + width;
-    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
-        const float s = item_score(L, ids[i], a.Ch, a.Cw, a.Ct);
-        const uint32_t u = ordered_key(s);
-        if (hi < 32 && (u >> hi) != (pre >> hi)) continue;
-        const int d = (int)((u >> shift) & (uint32_t)(nb - 1));
-        atomicAdd(&S.cnt[d], cnts[i]);
-        atomicAdd(&S.met[d], by_mass ? (unsigned long long)cnts[i] * item_mass(s, smax, a.inv_sqrt_d)
-                                     : (unsigned long long)cnts[i]);
-    }
-    __syncthreads();
-    // Buckets from the largest key down, blockDim at a time.
     for (int top = nb - 1; top >= 0; top -= blockDim.x) {
         const int b = top - (int)threadIdx.x;
         const unsigned long long v = b >= 0 ? S.met[b] : 0ull;
@@ -194,34 +237,59 @@ __device__ bool radix_pass(SelShared &S, const float *L, const int32_t *ids, con
         __syncthreads();
         if (S.bucket >= 0) break;
     }
-    const bool ok = S.bucket >= 0;
     __syncthreads();
-    if (threadIdx.x == 0 && ok) {
+    if (threadIdx.x == 0 && S.bucket >= 0) {
         S.above_met = S.new_above_met;
         S.above_cnt = S.new_above_cnt;
-        S.prefix = pre | ((uint32_t)S.bucket << shift);
     }
+    __syncthreads();
+}
+
+// One refine pass over `width` bits below `shift + width` of the order key,
+// among the items of coarse bucket S.coarse whose key matches S.prefix above.
+__device__ bool refine_pass(SelShared &S, const ItemKeys &K, const int32_t *cnts, int n_items, const CoarseMap &cm,
+                            float smax, float inv_sqrt_d, bool by_mass, unsigned long long target, int shift,
+                            int width)
+{
+    const int nb = 1 << width;
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        S.met[i] = 0ull;
+        S.cnt[i] = 0;
+    }
+    __syncthreads();
+    const uint32_t pre = S.prefix;
+    const int hi = shift + width, cb = S.coarse;
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const uint32_t u = K(i);
+        if (hi < 32 && (u >> hi) != (pre >> hi)) continue;
+        const float sc = key_score(u);
+        if (cm(sc) != cb) continue;
+        const int d = (int)((u >> shift) & (uint32_t)(nb - 1));
+        atomicAdd(&S.cnt[d], cnts[i]);
+        atomicAdd(&S.met[d], by_mass ? (unsigned long long)cnts[i] * item_mass(sc, smax, inv_sqrt_d)
+                                     : (unsigned long long)cnts[i]);
+    }
+    __syncthreads();
+    pick_bucket(S, nb, target);
+    const bool ok = S.bucket >= 0;
+    if (threadIdx.x == 0 && ok) S.prefix = pre | ((uint32_t)S.bucket << shift);
     __syncthreads();
     return ok;
 }
 
-// Finds the key at which the running metric (from the largest key down)
-// first reaches `target`.  Returns the number of keys taken: all keys above
-// that cut key plus `need` keys at it (-1 if the invariant broke).
-__device__ int radix_select(SelShared &S, const float *L, const int32_t *ids, const int32_t *cnts, int n_items,
-                            const SelArgs &a, float smax, bool by_mass, unsigned long long target,
-                            uint32_t *cut_key, int *need_at_cut)
+// After the coarse bucket is chosen (S.coarse, S.above_*): the exact order
+// key of the cut and the number of keys taken (-1 if the invariant broke,
+// which exact integer metrics rule out).
+__device__ int refine(SelShared &S, const ItemKeys &K, const int32_t *cnts, int n_items, const CoarseMap &cm,
+                      float smax, float inv_sqrt_d, bool by_mass, unsigned long long target, uint32_t *cut_key,
+                      int *need_at_cut)
 {
-    if (threadIdx.x == 0) {
-        S.prefix = 0u;
-        S.above_met = 0ull;
-        S.above_cnt = 0;
-    }
+    if (threadIdx.x == 0) S.prefix = 0u;
     __syncthreads();
-    if (!radix_pass(S, L, ids, cnts, n_items, a, smax, by_mass, target, 21, 11)) return -1;
-    if (!radix_pass(S, L, ids, cnts, n_items, a, smax, by_mass, target, 10, 11)) return -1;
-    if (!radix_pass(S, L, ids, cnts, n_items, a, smax, by_mass, target, 0, 10)) return -1;
-    // Every key in the final bucket has the same score, hence the same metric.
+    if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 21, 11)) return -1;
+    if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 10, 11)) return -1;
+    if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 0, 10)) return -1;
+    // every key in the final bucket has the same score, hence the same metric
     const unsigned long long per = S.bucket_met / (unsigned long long)S.bucket_cnt;
     const unsigned long long rest = target - S.above_met;
     const int need = (int)((rest + per - 1) / per);
@@ -230,51 +298,98 @@ __device__ int radix_select(SelShared &S, const float *L, const int32_t *ids, co
     return S.above_cnt + need;
 }
 
-__device__ float block_max_score(SelShared &S, const float *L, const int32_t *ids, int n_items, const SelArgs &a)
+// Order keys of the head's items (into the cache when there is one) and the
+// block's score range.
+__device__ void item_keys_and_range(SelShared &S, const float *L, const int32_t *ids, int n_items, uint32_t *cache,
+                                    int Ct, int Ch, int Cw, float *smin, float *smax)
 {
-    float m = -INFINITY;
-    for (int i = threadIdx.x; i < n_items; i += blockDim.x) m = fmaxf(m, item_score(L, ids[i], a.Ch, a.Cw, a.Ct));
-    m = warp_max(m);
-    if ((threadIdx.x & 31) == 0) S.fred[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        float v = threadIdx.x < (blockDim.x >> 5) ? S.fred[threadIdx.x] : -INFINITY;
-        v = warp_max(v);
-        if (threadIdx.x == 0) S.fred[0] = v;
+    float lo = INFINITY, hi = -INFINITY;
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const float sc = item_score(L, ids[i], Ch, Cw, Ct);
+        if (cache) cache[i] = ordered_key(sc);
+        lo = fminf(lo, sc);
+        hi = fmaxf(hi, sc);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        S.fmin[threadIdx.x >> 5] = lo;
+        S.fmax[threadIdx.x >> 5] = hi;
     }
     __syncthreads();
-    const float r = S.fred[0];
+    lo = INFINITY;
+    hi = -INFINITY;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        lo = fminf(lo, S.fmin[w]);
+        hi = fmaxf(hi, S.fmax[w]);
+    }
+    *smin = lo;
+    *smax = hi;
     __syncthreads();
-    return r;
 }
 
 // -------------------------------------------------------------- Top-p counts
-__global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r_out)
+__global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r_out, ClusterCut *cuts,
+                                                           int32_t *coarse_hist)
 {
-    extern __shared__ float L[];
+    extern __shared__ __align__(16) float L[];
     __shared__ SelShared S;
     const int c = blockIdx.x, bh = blockIdx.y;
+    const int64_t bhc = (int64_t)bh * a.Cq + c;
     const int Csum = a.Ct + a.Ch + a.Cw;
-    const float *lrow = a.lut + ((int64_t)bh * a.Cq + c) * Csum;
+    uint32_t *cache = reinterpret_cast<uint32_t *>(L + ((Csum + 3) & ~3));
+    const float *lrow = a.lut + bhc * Csum;
     for (int e = threadIdx.x; e < Csum; e += blockDim.x) L[e] = lrow[e];
     __syncthreads();
     const int n_items = a.item_n[bh];
     const int32_t *ids = a.item_id + (int64_t)bh * a.Pcap;
     const int32_t *cnts = a.item_cnt + (int64_t)bh * a.Pcap;
+    if (n_items > kItemCache) cache = nullptr;
+    float smin, smax;
+    item_keys_and_range(S, L, ids, n_items, cache, a.Ct, a.Ch, a.Cw, &smin, &smax);
+    const ItemKeys K{cache, L, ids, a.Ct, a.Ch, a.Cw};
+    const CoarseMap cm(smin, smax);
     int m = a.N;
-    if (a.top_p < 1.0f) {
-        const float smax = block_max_score(S, L, ids, n_items, a);
-        unsigned long long W = 0ull;
-        for (int i = threadIdx.x; i < n_items; i += blockDim.x)
-            W += (unsigned long long)cnts[i] * item_mass(item_score(L, ids[i], a.Ch, a.Cw, a.Ct), smax, a.inv_sqrt_d);
+    uint32_t key = 0u;
+    int need = 0;
+    // coarse histogram by count and by mass, over every item
+    for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) {
+        S.met[i] = 0ull;
+        S.cnt[i] = 0;
+    }
+    __syncthreads();
+    const bool sel = a.top_p < 1.0f;
+    unsigned long long wsum = 0ull;
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const float sc = key_score(K(i));
+        const int b = cm(sc);
+        atomicAdd(&S.cnt[b], cnts[i]);
+        if (sel) {
+            const unsigned long long w = (unsigned long long)cnts[i] * item_mass(sc, smax, a.inv_sqrt_d);
+            atomicAdd(&S.met[b], w);
+            wsum += w;
+        }
+    }
+    __syncthreads();
+    int32_t *hist_out = coarse_hist + bhc * kBuckets;
+    for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) hist_out[i] = S.cnt[i];
+    if (sel) {
         unsigned long long Wt;
-        block_excl_scan(W, S.utmp, Wt);
+        block_excl_scan(wsum, S.utmp, Wt);
         unsigned long long target = (unsigned long long)ceil((double)a.top_p * (double)Wt);
         if (target < 1ull) target = 1ull;
         if (target > Wt) target = Wt;
-        uint32_t key;
-        int need;
-        m = radix_select(S, L, ids, cnts, n_items, a, smax, true, target, &key, &need);
+        if (threadIdx.x == 0) {
+            S.above_met = 0ull;
+            S.above_cnt = 0;
+        }
+        __syncthreads();
+        pick_bucket(S, kBuckets, target);
+        if (threadIdx.x == 0) S.coarse = S.bucket;
+        __syncthreads();
+        m = S.coarse >= 0 ? refine(S, K, cnts, n_items, cm, smax, a.inv_sqrt_d, true, target, &key, &need) : -1;
         if (m < 0) {
             if (threadIdx.x == 0) set_error(a.err, kErrRange, 0x100 + c);
             m = a.N;
@@ -283,7 +398,15 @@ __global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r
     if (threadIdx.x == 0) {
         int r = m > a.k_min ? m : a.k_min;
         r = r < a.N ? r : a.N;
-        r_out[(int64_t)bh * a.Cq + c] = r;
+        r_out[bhc] = r;
+        ClusterCut cut;
+        cut.smin = smin;
+        cut.smax = smax;
+        cut.key = key;
+        cut.need = need;
+        cut.taken = sel ? m : a.N;
+        cut.pad[0] = cut.pad[1] = cut.pad[2] = 0;
+        cuts[bhc] = cut;
     }
 }
 
@@ -324,15 +447,19 @@ __global__ void __launch_bounds__(1024) topk_kernel(const int32_t *sizes, const 
 
 // -------------------------------------------------------------- list emission
 // The first n_c keys of the (score desc, index asc) order: every key strictly
-// above the cut score, then the lowest-index `need` keys at the cut score.
-// Written in ascending key order: the output slot of key j is
+// above the cut, then the lowest-index `need` keys at the cut.  When n_c is
+// the cluster's Top-p count the cut is the Top-p kernel's; otherwise a count
+// select runs from that kernel's coarse histogram.  Written in ascending key
+// order: the output slot of key j is
 // (#keys above the cut before j) + min(#keys at the cut before j, need).
-// A key's side of the cut is its item's, so the items are classed once in
-// shared memory (2 above, 1 at, 0 below) and each key costs one 16-bit load.
+// A key's side of the cut is its item's: each key costs one 16-bit load of its
+// item rank and one shared-memory lookup (the item's order key, or a class
+// byte when the keys are not cached).
 constexpr int kEmitPer = 8;
 
-__global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int32_t *n_in,
-                                                           const long long *offsets, int32_t *indices)
+__global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int32_t *n_in, const long long *offsets,
+                                                           const ClusterCut *cuts, const int32_t *coarse_hist,
+                                                           int32_t *indices)
 {
     extern __shared__ __align__(16) float L[];
     __shared__ SelShared S;
@@ -347,24 +474,62 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         return;
     }
     const int Csum = a.Ct + a.Ch + a.Cw;
-    uint8_t *cls = reinterpret_cast<uint8_t *>(L + ((Csum + 3) & ~3));
+    unsigned char *region = reinterpret_cast<unsigned char *>(L + ((Csum + 3) & ~3));  // 64 KB
     const float *lrow = a.lut + bhc * Csum;
     for (int e = threadIdx.x; e < Csum; e += blockDim.x) L[e] = lrow[e];
     __syncthreads();
     const int n_items = a.item_n[bh];
     const int32_t *ids = a.item_id + (int64_t)bh * a.Pcap;
     const int32_t *cnts = a.item_cnt + (int64_t)bh * a.Pcap;
-    uint32_t cut;
-    int need;
-    if (radix_select(S, L, ids, cnts, n_items, a, 0.f, false, (unsigned long long)n, &cut, &need) < 0) {
-        if (threadIdx.x == 0) set_error(a.err, kErrRange, 0x200 + c);
-        return;
+    const bool cached = n_items <= kItemCache;
+    uint32_t *cache = cached ? reinterpret_cast<uint32_t *>(region) : nullptr;
+    if (cached)
+        for (int i = threadIdx.x; i < n_items; i += blockDim.x)
+            cache[i] = ordered_key(item_score(L, ids[i], a.Ch, a.Cw, a.Ct));
+    __syncthreads();
+    const ItemKeys K{cache, L, ids, a.Ct, a.Ch, a.Cw};
+    const ClusterCut cut = cuts[bhc];
+    uint32_t key = cut.key;
+    int need = cut.need;
+    if (n != cut.taken) {
+        // count select for n: coarse bucket from the stored histogram, then refine
+        const int32_t *hist = coarse_hist + bhc * kBuckets;
+        for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) {
+            const int k = hist[i];
+            S.cnt[i] = k;
+            S.met[i] = (unsigned long long)k;
+        }
+        if (threadIdx.x == 0) {
+            S.above_met = 0ull;
+            S.above_cnt = 0;
+        }
+        __syncthreads();
+        pick_bucket(S, kBuckets, (unsigned long long)n);
+        if (threadIdx.x == 0) S.coarse = S.bucket;
+        __syncthreads();
+        const CoarseMap cm(cut.smin, cut.smax);
+        if (S.coarse < 0 ||
+            refine(S, K, cnts, n_items, cm, cut.smax, a.inv_sqrt_d, false, (unsigned long long)n, &key, &need) < 0) {
+            if (threadIdx.x == 0) set_error(a.err, kErrRange, 0x200 + c);
+            return;
+        }
     }
-    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
-        const uint32_t u = ordered_key(item_score(L, ids[i], a.Ch, a.Cw, a.Ct));
-        cls[i] = u > cut ? 2 : (u == cut ? 1 : 0);
+    // without cached keys, class every item once: 2 above, 1 at, 0 below the cut
+    uint8_t *cls = region;
+    if (!cached) {
+        for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+            const uint32_t u = K(i);
+            cls[i] = u > key ? 2 : (u == key ? 1 : 0);
+        }
     }
     __syncthreads();
+    auto class_of = [&](int item) -> uint8_t {
+        if (cached) {
+            const uint32_t u = cache[item];
+            return u > key ? 2 : (u == key ? 1 : 0);
+        }
+        return cls[item];
+    };
     const uint16_t *ki = a.key_item + (int64_t)bh * a.N;
     const bool vec = (((int64_t)bh * a.N) & 7) == 0;  // 16-byte aligned rows of 8 ranks
     int gt_run = 0, eq_run = 0;
@@ -376,10 +541,10 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
             const uint4 w = *reinterpret_cast<const uint4 *>(ki + j0);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int t = 0; t < kEmitPer; ++t) k[t] = cls[(ws[t >> 1] >> (16 * (t & 1))) & 0xffffu];
+            for (int t = 0; t < kEmitPer; ++t) k[t] = class_of((ws[t >> 1] >> (16 * (t & 1))) & 0xffffu);
         } else {
 #pragma unroll
-            for (int t = 0; t < kEmitPer; ++t) k[t] = j0 + t < a.N ? cls[ki[j0 + t]] : 0;
+            for (int t = 0; t < kEmitPer; ++t) k[t] = j0 + t < a.N ? class_of(ki[j0 + t]) : 0;
         }
 #pragma unroll
         for (int t = 0; t < kEmitPer; ++t) {
@@ -410,12 +575,18 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
     }
 }
 
-static size_t emit_smem(int Csum, int Pcap) { return (size_t)((Csum + 3) & ~3) * sizeof(float) + (size_t)Pcap; }
+// dynamic shared memory of topp_kernel and emit_kernel: the table row and a
+// 64 KB region (cached order keys, or item class bytes)
+static size_t sel_smem(int Csum) { return (size_t)((Csum + 3) & ~3) * sizeof(float) + (size_t)kItemCache * 4; }
 
 cudaError_t select_configure()
 {
-    return cudaFuncSetAttribute(emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)emit_smem(3 * kMaxClusters, kMaxItems));
+    static_assert(kItemCache * 4 >= kMaxItems, "the 64 KB region must hold a class byte per item");
+    cudaError_t e = cudaFuncSetAttribute(emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sel_smem(3 * kMaxClusters));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(topp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sel_smem(3 * kMaxClusters));
 }
 
 // -------------------------------------------------------------- launchers
@@ -439,10 +610,9 @@ void launch_items(const int32_t *codes, int32_t *hist, int32_t *item_id, int32_t
     count_launches(1);
 }
 
-void launch_topp(const SelArgs &a, int32_t *r_out, cudaStream_t st)
+void launch_topp(const SelArgs &a, int32_t *r_out, ClusterCut *cuts, int32_t *coarse_hist, cudaStream_t st)
 {
-    const size_t smem = (size_t)(a.Ct + a.Ch + a.Cw) * sizeof(float);
-    topp_kernel<<<dim3(a.Cq, a.BH), kSelThreads, smem, st>>>(a, r_out);
+    topp_kernel<<<dim3(a.Cq, a.BH), kSelThreads, sel_smem(a.Ct + a.Ch + a.Cw), st>>>(a, r_out, cuts, coarse_hist);
     count_launches(1);
 }
 
@@ -453,18 +623,22 @@ void launch_topk(const int32_t *sizes, const int32_t *r, int32_t *n_out, int32_t
     count_launches(1);
 }
 
-void launch_emit(const SelArgs &a, const int32_t *n_in, const long long *offsets, int32_t *indices, cudaStream_t st)
+void launch_emit(const SelArgs &a, const int32_t *n_in, const long long *offsets, const ClusterCut *cuts,
+                 const int32_t *coarse_hist, int32_t *indices, cudaStream_t st)
 {
-    const size_t smem = emit_smem(a.Ct + a.Ch + a.Cw, a.Pcap);
-    emit_kernel<<<dim3(a.Cq, a.BH), kSelThreads, smem, st>>>(a, n_in, offsets, indices);
+    emit_kernel<<<dim3(a.Cq, a.BH), kSelThreads, sel_smem(a.Ct + a.Ch + a.Cw), st>>>(a, n_in, offsets, cuts,
+                                                                                  coarse_hist, indices);
     count_launches(1);
 }
+
+// Bytes of per-cluster selection state (cut record + coarse histogram).
+size_t selection_state_bytes(int64_t clusters) { return (size_t)clusters * (sizeof(ClusterCut) + kBuckets * 4); }
 
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
                    const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch,
                    int Cw, int BH, float top_p, float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes,
                    int32_t *r, int32_t *n, int32_t *kh, long long *offsets, int32_t *indices, int online,
-                   cudaStream_t st)
+                   void *state, cudaStream_t st)
 {
     SelArgs a;
     a.lut = lut;
@@ -484,9 +658,11 @@ void run_selection(const float *lut, const int32_t *codes, const int32_t *item_i
     a.inv_sqrt_d = inv_sqrt_d;
     a.k_min = k_min;
     a.err = err;
-    launch_topp(a, r, st);
+    ClusterCut *cuts = reinterpret_cast<ClusterCut *>(state);
+    int32_t *coarse_hist = reinterpret_cast<int32_t *>(cuts + (int64_t)BH * Cq);
+    launch_topp(a, r, cuts, coarse_hist, st);
     launch_topk(sizes, r, n, kh, offsets, BH, Cq, N, online, st);
-    launch_emit(a, n, offsets, indices, st);
+    launch_emit(a, n, offsets, cuts, coarse_hist, indices, st);
 }
 
 }  // namespace scope

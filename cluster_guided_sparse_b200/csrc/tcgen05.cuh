@@ -37,9 +37,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait: false after ~2 s or once another thread of the CTA aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          int32_t *err, int where)
+// Bounded wait: false after `limit` SM clock cycles (recording the timeout
+// bit and `where` in the device error word and raising the CTA's abort flag),
+// or once another thread of the CTA aborted.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                int32_t *err, int where, long long limit)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
@@ -47,13 +49,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 255u) == 0u) {
             if (*abort_flag) return false;
-            if (clock64() - t0 > kWaitCycles) {
+            if (clock64() - t0 > limit) {
                 *abort_flag = 1;
                 set_error(err, kErrTimeout, where);
                 return false;
             }
         }
     }
+}
+
+// The kernels' wait: gives up after ~2 s.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *err, int where)
+{
+    return mbar_wait_limit(bar, parity, abort_flag, err, where, kWaitCycles);
 }
 
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)

@@ -101,6 +101,17 @@ WORKLOADS = {
         components=128, sigma=(0.1, 1.0), zipf_alpha=0.0,
         d_split=(16, 56, 56), theta=10000.0, c_q=512, c_sub=(16, 32, 32), iters=10,
         top_p=0.9, k_min=0, online_topk=1, fixed_cluster_size=0),
+    # The same layer with spatially coherent content: tokens of one 11x15x16
+    # grid block share a component label (objects occupying regions), which
+    # the proxy scores resolve far more sharply than i.i.d. labels.  A second,
+    # separately labelled measurement; the 720p line above stays the headline.
+    "hunyuan720p_regions": Workload(
+        name="HunyuanVideo-720p-shaped layer, region-coherent content (B=1,H=24,d=128, grid 33x45x80, "
+             "N=118800, bf16, labels shared by 11x15x16 blocks)",
+        config_id=6, B=1, H=24, N=118800, D=128, grid=(33, 45, 80), dtype="bf16",
+        components=128, sigma=(0.1, 1.0), zipf_alpha=0.0,
+        d_split=(16, 56, 56), theta=10000.0, c_q=512, c_sub=(16, 32, 32), iters=10,
+        top_p=0.9, k_min=0, online_topk=1, fixed_cluster_size=0, label_block=(11, 15, 16)),
     "unstructured": Workload(
         name="unstructured bidirectional variant (B=1,H=6,d=64, N=65536, no grid, bf16)",
         config_id=5, B=1, H=6, N=65536, D=64, grid=(0, 0, 0), dtype="bf16",

@@ -8,8 +8,9 @@
  *    (abstract: power-of-two cluster sizes, block-sparse attention).
  *
  * Conventions for every entry point
- *   - Tensors are DEVICE memory owned by the caller, contiguous row-major
- *     [B, H, N, D] (D fastest), 16-byte aligned.  D is 64 or 128.
+ *   - Tensors are DEVICE memory owned by the caller, logical shape
+ *     [B, H, N, D] (D is 64 or 128) with element strides (see scope_tensor);
+ *     every row of D elements is contiguous and starts on a 16-byte boundary.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  All device work is enqueued on it; no call synchronises the
  *     host except scope_sync_status.
@@ -51,11 +52,22 @@ typedef enum {
     SCOPE_I64 = 3
 } scope_dtype;
 
-/* A caller-owned device tensor, contiguous [B, H, N, D]. */
+/* A caller-owned device tensor of logical shape [B, H, N, D].
+ *   strides  element strides of the B, H, N and D dimensions.  strides[3]
+ *            must be 1 (a row of D elements is contiguous); strides[0..2]
+ *            must be >= 0 and keep every row start 16-byte aligned
+ *            (multiples of 8 elements for bf16, of 4 for f32), and distinct
+ *            (b, h, n) must not share a row.  All four zero means the
+ *            contiguous layout {H*N*D, N*D, D, 1}.  Any other layout (for
+ *            example [B, N, H, D] memory seen as [B, H, N, D], or every
+ *            second head of a larger tensor) is read and written in place.
+ *            scope_kmeans_noalloc takes contiguous x only.
+ *   A layout outside these rules returns SCOPE_ESHAPE before any launch. */
 typedef struct {
     void *ptr;
     scope_dtype dtype;
     int64_t B, H, N, D;
+    int64_t strides[4];
 } scope_tensor;
 
 /* Latent grid of the tokens: token n sits at (t, y, x) with
@@ -193,6 +205,16 @@ scope_status scope_plan_view(const scope_plan_t *plan, int which, scope_view *ou
  * SCOPE_ECUDA (an asynchronous CUDA error). */
 scope_status scope_sync_status(const scope_plan_t *plan, void *stream);
 
+/* Failure-handling self-test (no counterpart on the pages).  Enqueues one
+ * CTA that waits, with the same bounded mbarrier wait every tensor-core
+ * kernel of the library uses, on a barrier nothing ever arrives on; after
+ * `wait_cycles` SM clock cycles (1e3 .. 4e9; 2e6 is about a millisecond) the
+ * wait gives up and sets the timeout bit of the plan's device error word,
+ * as a stalled kernel would.  scope_sync_status(plan) then returns
+ * SCOPE_ETIMEOUT.  Nothing faults or hangs and the CUDA context stays
+ * usable; the plan's error word stays set (make a new plan to clear it). */
+scope_status scope_selftest_wait_timeout(const scope_plan_t *plan, int64_t wait_cycles, void *stream);
+
 /* Frees the host handle only; the workspace stays the caller's. */
 void scope_plan_destroy(scope_plan_t *plan);
 
@@ -209,10 +231,16 @@ int scope_version(void);
 /* memory plan is fixed after start-up, a plug-in that may only touch the   */
 /* buffers its host passes in).                                             */
 /*                                                                          */
-/* scope_kmeans_noalloc runs the same Lloyd k-means as scope_plan's step 2  */
-/* on columns [dim_off, dim_off + dim_n) of x, with the same strided init,  */
-/* tie rule, empty-cluster rule and final assign, so its results equal the  */
-/* plan's for the same rows.                                                */
+/* scope_kmeans_noalloc runs Lloyd k-means on columns                      */
+/* [dim_off, dim_off + dim_n) of x with scope_plan's strided init, tie      */
+/* rule, empty-cluster rule, final assign and per-head fixed-point centroid */
+/* sums, assigning by the fp32 direct-form distance.  Given the plan's      */
+/* rotated rows and C < 128 (the plan's key subspaces, and its queries at   */
+/* fewer than 128 clusters) its labels and centroids equal the plan's.  At  */
+/* C >= 128 the plan decides query labels exactly (tensor cores plus an     */
+/* fp64 re-decision of near-ties), while this entry point keeps the fp32    */
+/* direct form: a label can then differ where a row's two nearest centroids */
+/* lie within fp32 rounding of each other, and later rounds follow from it. */
 /*   x          bf16 [B,H,N,D] device, D in {64, 128} (e.g. post-RoPE rows). */
 /*   labels     int32 [B,H,N] device, written (final assign).               */
 /*   centroids  f32 [B,H,C,dim_n] device, written (after the last update).  */

@@ -142,3 +142,38 @@ def test_compensation_workspace_holds_row_lse_and_cluster_means(L):
         sizes.append(L.scope_plan_workspace_bytes(ctypes.byref(q), ctypes.byref(g), ctypes.byref(p)))
     BH, N, C, D = 2, 4096, 64, 64
     assert sizes[0] > 0 and sizes[1] >= sizes[0] + BH * N * 4 + BH * C * D * 4
+
+
+def S(strides, N=256, D=64, H=2, B=1, dtype=scope.SCOPE_BF16):
+    return scope.ScopeTensor(FAKE, dtype, B, H, N, D, (ctypes.c_int64 * 4)(*strides))
+
+
+def test_strided_layouts_checked_on_host(L):
+    p, g = P()
+    N, D, H = 256, 64, 2
+    ws_of = lambda t: L.scope_plan_workspace_bytes(ctypes.byref(t), ctypes.byref(g), ctypes.byref(p))
+    contiguous = ws_of(T())
+    # accepted: explicit contiguous strides, [B, N, H, D] memory, every second head of a 4-head tensor
+    for st in ((H * N * D, N * D, D, 1), (N * H * D, D, H * D, 1), (4 * N * D, 2 * N * D, D, 1)):
+        assert ws_of(S(st)) == contiguous, st
+    # rejected before any device work: D not contiguous, misaligned row starts, rows that overlap
+    for st, msg in (((H * N * D, N * D, D, 2), "strides[3]"), ((H * N * D, N * D, 68, 1), "16 bytes"),
+                    ((H * N * D, N * D, 32, 1), "overlap"), ((N * D, 0, D, 1), "overlap"),
+                    ((H * N * D, -N * D, D, 1), ">= 0")):
+        q = S(st)
+        assert plan_status(L, q, q, p, g)[0] == 2, st
+        assert msg in L.scope_last_error().decode(), (st, L.scope_last_error())
+    # f32 rows need 16-byte alignment too: a stride of 4 floats is fine, 2 is not
+    p32 = S((H * N * 68, N * 68, 68, 1), dtype=scope.SCOPE_F32)
+    assert ws_of(p32) == ws_of(T(dtype=scope.SCOPE_F32))
+    bad = S((H * N * 66, N * 66, 66, 1), dtype=scope.SCOPE_F32)
+    assert plan_status(L, bad, bad, p, g)[0] == 2
+
+
+def test_selftest_wait_timeout_checks_arguments(L):
+    L.scope_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+    assert L.scope_selftest_wait_timeout(None, 2_000_000, None) == 1
+    # the cycle limit is checked before the plan is touched (fake handle)
+    assert L.scope_selftest_wait_timeout(ctypes.c_void_p(FAKE), 10, None) == 1
+    assert "wait_cycles" in L.scope_last_error().decode()
+    assert L.scope_selftest_wait_timeout(ctypes.c_void_p(FAKE), 5_000_000_000, None) == 1

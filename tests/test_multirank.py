@@ -1,8 +1,9 @@
 """Multi-rank logic of bench.py on CPU: two gloo ranks (world size 2).
 
-bench.py runs one process per GPU under torchrun; the rank-level pieces it
-relies on are the barrier, the max of a per-rank time over all ranks, the
-whole-job ms-per-call and the rank-0-only reference line.  They are checked
+bench.py runs one process per GPU under torchrun, one call's heads split
+round-robin over the ranks; the rank-level pieces it relies on are the
+barrier, the max and sum of per-rank values over all ranks, the ms per call,
+the rank-0-only reference line and the head-sharded call itself.  They are checked
 here with a gloo process group on 127.0.0.1, no GPU involved.
 """
 import json
@@ -37,10 +38,11 @@ def _worker(rank, world, port, out_dir):
         bench.barrier(world)
         # rank r "measured" 10 * (r + 1) ms for its steps
         mx = bench.max_over_ranks(10.0 * (rank + 1), world)
-        per_call = bench.job_ms_per_call(10.0 * (rank + 1), 5, world)
+        per_call = bench.call_ms(10.0 * (rank + 1), 5, world)
+        total = bench.sum_over_ranks(1.0 + rank, world)
         bench.barrier(world)
         with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
-            json.dump({"max": mx, "per_call": per_call}, f)
+            json.dump({"max": mx, "per_call": per_call, "sum": total}, f)
     finally:
         dist.destroy_process_group()
 
@@ -53,7 +55,8 @@ def test_two_gloo_ranks_agree_on_max_and_job_rate(tmp_path):
     res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
     for r in res:
         assert r["max"] == 20.0  # the slowest rank's time, on every rank
-        assert r["per_call"] == pytest.approx(20.0 / (5 * 2))  # 5 calls per rank, 2 ranks
+        assert r["per_call"] == pytest.approx(20.0 / 5)  # 5 calls, each spread over both ranks
+        assert r["sum"] == 3.0
 
 
 def test_single_rank_needs_no_process_group():
@@ -63,7 +66,8 @@ def test_single_rank_needs_no_process_group():
     assert not dist.is_initialized()
     bench.barrier(1)
     assert bench.max_over_ranks(3.5, 1) == 3.5
-    assert bench.job_ms_per_call(30.0, 3, 1) == pytest.approx(10.0)
+    assert bench.call_ms(30.0, 3, 1) == pytest.approx(10.0)
+    assert bench.sum_over_ranks(2.5, 1) == 2.5
 
 
 def test_reference_arm_prints_nothing_off_rank0(capsys):
@@ -102,3 +106,86 @@ def test_reference_arm_line_has_the_contract_keys(capsys):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+# --------------------------------------------------------------------------- head sharding
+def _host_scope_heads(q, k, v, params, grid):
+    """Per-head SCOPE call on the host (the oracle), standing in for the
+    library on gloo ranks that have no GPU: [B, H', N, D] float64 output."""
+    import numpy as np
+
+    import oracle
+
+    p = params
+    B, Hl, N, D = q.shape
+    out = torch.empty((B, Hl, N, D), dtype=torch.float64)
+    for b in range(B):
+        for h in range(Hl):
+            pl = oracle.scope_plan_head(q[b, h].double().numpy(), k[b, h].double().numpy(), p)
+            o = oracle.scope_attn_head(pl["qr"], pl["kr"], v[b, h].double().numpy(), pl["q_labels"], pl["lists"])
+            out[b, h] = torch.from_numpy(np.ascontiguousarray(o))
+    return out
+
+
+def _shard_worker(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+
+    import oracle
+    from cluster_guided_sparse_b200 import shard, synth
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = synth.WORKLOADS["tiny"].with_(H=3)  # 3 heads over 2 ranks: {0, 2} and {1}
+        q, k, v = synth.make_inputs(w)
+        p = oracle.Params.of(w)
+        local = shard.sharded_attention(q, k, v, p, None, gather=False, run=_host_scope_heads)
+        full = shard.sharded_attention(q, k, v, p, None, run=_host_scope_heads)
+        # a rank that holds only its own heads (pass the total head count)
+        mine = shard.heads_of(w.H, rank, world)
+        own = shard.sharded_attention(q[:, mine], k[:, mine], v[:, mine], p, None, H=w.H,
+                                      run=_host_scope_heads)
+        torch.save({"local": local, "full": full, "own": own, "heads": mine},
+                   os.path.join(out_dir, f"shard{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_head_sharded_call_equals_single_rank(tmp_path):
+    sys.path.insert(0, ROOT)
+    import oracle
+    from cluster_guided_sparse_b200 import shard, synth
+
+    world = 2
+    mp.start_processes(_shard_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    w = synth.WORKLOADS["tiny"].with_(H=3)
+    q, k, v = synth.make_inputs(w)
+    ref = shard.sharded_attention(q, k, v, oracle.Params.of(w), None, run=_host_scope_heads)  # no group: 1 rank
+    seen = []
+    for r in range(world):
+        res = torch.load(tmp_path / f"shard{r}.pt")
+        assert res["heads"] == shard.heads_of(3, r, world) == [h for h in range(3) if h % world == r]
+        assert torch.equal(res["local"], ref[:, res["heads"]])  # each rank computed exactly its heads
+        assert torch.equal(res["full"], ref)  # the all-gather reassembles every head in place
+        assert torch.equal(res["own"], ref)
+        seen += res["heads"]
+    assert sorted(seen) == [0, 1, 2]
+
+
+def test_head_partition_rules():
+    sys.path.insert(0, ROOT)
+    from cluster_guided_sparse_b200 import shard
+
+    for H in (1, 3, 24, 40):
+        for world in (1, 2, 3, 8):
+            parts = [shard.heads_of(H, r, world) for r in range(world)]
+            assert sorted(h for p in parts for h in p) == list(range(H))
+            assert max(map(len, parts)) - min(map(len, parts)) <= 1
+    x = torch.arange(2 * 5 * 3 * 4, dtype=torch.float32).view(2, 5, 3, 4)
+    assert torch.equal(shard.local_heads(x, 1, 2), x[:, [1, 3]])
+    with pytest.raises(ValueError):
+        shard.heads_of(4, 2, 2)
