@@ -76,6 +76,10 @@ def lib():
         L.orc_bisect.argtypes = [_d, _I, _I, _I, ctypes.c_int, _i32, _d, _i64]
         L.orc_attn_rows_comp.argtypes = [_d, _I, _d, _d, _I, _I, _i32, _I, _i32, _I, ctypes.c_double, _d]
         L.orc_bisect.restype = ctypes.c_int
+        L.orc_head_entropy.argtypes = [_d, _i64, _I, _I, ctypes.c_double]
+        L.orc_head_entropy.restype = ctypes.c_double
+        L.orc_pooled_topp.argtypes = [_d, _i64, _I, _I, _I, ctypes.c_double, ctypes.c_double, _i64]
+        L.orc_pooled_topp.restype = ctypes.c_double
         _lib = L
     return _lib
 
@@ -198,6 +202,55 @@ def emit(s, n: int) -> np.ndarray:
     out = np.empty(int(n), np.int32)
     lib().orc_emit(s, s.shape[0], int(n), out)
     return out
+
+
+def head_entropy(scores, sizes, scale: float) -> float:
+    """EG-Sparse head entropy: query-size-weighted mean row entropy of the
+    proxy softmax, over ln N (R17).  scores [C, N], sizes [C]."""
+    sc = _f64(scores)
+    C, N = sc.shape
+    return lib().orc_head_entropy(sc, np.ascontiguousarray(sizes, np.int64), C, N, float(scale))
+
+
+def pooled_topp(scores, sizes, p: float, scale: float, with_mass: bool = False):
+    """EG-Sparse pooled Top-p counts of one pool of heads (R17).
+    scores [Hp, C, N], sizes [Hp, C] -> counts [Hp, C] (and the kept mass fraction)."""
+    sc = _f64(scores)
+    Hp, C, N = sc.shape
+    counts = np.empty((Hp, C), np.int64)
+    mass = lib().orc_pooled_topp(sc, np.ascontiguousarray(sizes, np.int64), Hp, C, N, float(p), float(scale),
+                                 counts)
+    return (counts, mass) if with_mass else counts
+
+
+def eg_route(entropies, tau: float, group: int):
+    """Pools of one batch entry: for each group of `group` consecutive heads,
+    the list of its heads whose entropy is below tau (R17)."""
+    H = len(entropies)
+    pools = []
+    for g0 in range(0, H, group):
+        pools.append([h for h in range(g0, min(H, g0 + group)) if entropies[h] < tau])
+    return pools
+
+
+def eg_counts(scores_heads, sizes_heads, p: float, tau: float, group: int, scale: float):
+    """EG-Sparse Top-p counts of one batch entry's heads (R17).
+    scores_heads: per head [C, N] proxy scores; sizes_heads: per head [C].
+    Returns (entropies [H], pools, counts [H, C]): pooled heads take their
+    counts from their pool, the others from their own rows."""
+    H = len(scores_heads)
+    ent = [head_entropy(s, z, scale) for s, z in zip(scores_heads, sizes_heads)]
+    pools = eg_route(ent, tau, group)
+    C, N = np.asarray(scores_heads[0]).shape
+    counts = np.empty((H, C), np.int64)
+    for h in range(H):
+        for c in range(C):
+            counts[h, c] = topp_count(scores_heads[h][c], p, scale) if p < 1.0 else N
+    for pool in pools:
+        if pool:
+            counts[pool] = pooled_topp(np.stack([scores_heads[h] for h in pool]),
+                                       np.stack([sizes_heads[h] for h in pool]), p, scale)
+    return ent, pools, counts
 
 
 def attention_rows(q_rows, K, V, sel, scale: float) -> np.ndarray:

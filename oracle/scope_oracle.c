@@ -276,6 +276,114 @@ int64_t orc_online_topk(const int64_t *sizes, const int64_t *r, int64_t C,
     return online ? K : 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* EG-Sparse ["EG-Sparse", abstract: low-entropy heads are routed to a       */
+/* grouped cross-head pool, high-entropy heads keep per-row selection, using */
+/* only scores the sparse pipeline already has].  Readings (R17):           */
+/*  - a row is a query cluster c of head h; its proxy distribution is        */
+/*    pi_c(j) = softmax_j(scale * s_c(j)) over all N keys;                   */
+/*  - head entropy E_h = sum_c |c| H(pi_c) / (sum_c |c| * ln N), H in nats,  */
+/*    so 0 <= E_h <= 1 (1: uniform rows);                                    */
+/*  - head h is low-entropy iff E_h < tau; heads are grouped G at a time in  */
+/*    index order, and a group's low-entropy heads form one pool;           */
+/*  - in a pool every (h, c, j) competes at once: entries ranked by pi_c(j)  */
+/*    descending (ties: h, then c, then the row's own key order), each       */
+/*    carrying mass |c| pi_c(j); the shortest prefix reaching p of the       */
+/*    pool's total mass (sum over its heads of sum_c |c|) is kept, and       */
+/*    |P_c| = the number of kept entries of row c -- a prefix of that row's  */
+/*    own key order, so lists, k_min and the online Top-k follow as before.  */
+/* ------------------------------------------------------------------------ */
+
+/* Normalised entropy of one head: s [C][N] proxy scores, sizes [C]. */
+double orc_head_entropy(const double *s, const int64_t *sizes, int64_t C, int64_t N, double scale)
+{
+    if (N <= 1) return 0.0;
+    double num = 0.0, den = 0.0;
+    for (int64_t c = 0; c < C; ++c) {
+        if (sizes[c] <= 0) continue;
+        const double *sc = s + c * N;
+        double mx = sc[0];
+        for (int64_t j = 1; j < N; ++j) mx = sc[j] > mx ? sc[j] : mx;
+        double Z = 0.0;
+        for (int64_t j = 0; j < N; ++j) Z += exp((sc[j] - mx) * scale);
+        double H = 0.0;
+        for (int64_t j = 0; j < N; ++j) {
+            const double pj = exp((sc[j] - mx) * scale) / Z;
+            if (pj > 0.0) H -= pj * log(pj);
+        }
+        num += (double)sizes[c] * H;
+        den += (double)sizes[c];
+    }
+    return den > 0.0 ? num / (den * log((double)N)) : 0.0;
+}
+
+typedef struct {
+    double logp;     /* ln pi of the entry */
+    double mass;     /* |c| pi */
+    int64_t h, c, pos; /* pool head, row, place in the row's own order */
+} pool_entry;
+
+static int cmp_pool(const void *pa, const void *pb)
+{
+    const pool_entry *a = (const pool_entry *)pa, *b = (const pool_entry *)pb;
+    if (a->logp > b->logp) return -1;
+    if (a->logp < b->logp) return 1;
+    if (a->h != b->h) return (a->h > b->h) - (a->h < b->h);
+    if (a->c != b->c) return (a->c > b->c) - (a->c < b->c);
+    return (a->pos > b->pos) - (a->pos < b->pos);
+}
+
+/* Pooled Top-p counts of one pool: s [Hp][C][N] proxy scores of the pool's
+ * heads, sizes [Hp][C]; counts [Hp][C] receives |P_c| (N when p >= 1).  A
+ * cluster with no queries has no rows to pool: it keeps its own per-row
+ * Top-p count.  Returns the kept mass fraction (for near-tie accounting). */
+double orc_pooled_topp(const double *s, const int64_t *sizes, int64_t Hp, int64_t C, int64_t N, double p,
+                       double scale, int64_t *counts)
+{
+    int64_t E = 0;
+    for (int64_t i = 0; i < Hp * C; ++i) {
+        counts[i] = p >= 1.0 ? N : 0;
+        if (sizes[i] > 0) E += N;
+        else if (p < 1.0) counts[i] = orc_topp_count(s + i * N, N, p, scale, NULL);
+    }
+    if (p >= 1.0 || E == 0) return 1.0;
+    pool_entry *e = (pool_entry *)malloc((size_t)E * sizeof(pool_entry));
+    int64_t *order = (int64_t *)malloc((size_t)N * sizeof(int64_t));
+    double total = 0.0;
+    int64_t m = 0;
+    for (int64_t h = 0; h < Hp; ++h)
+        for (int64_t c = 0; c < C; ++c) {
+            if (sizes[h * C + c] <= 0) continue;
+            const double *sc = s + (h * C + c) * N;
+            orc_order(sc, N, order);
+            const double mx = sc[order[0]];
+            double Z = 0.0;
+            for (int64_t j = 0; j < N; ++j) Z += exp((sc[j] - mx) * scale);
+            const double lnZ = log(Z);
+            for (int64_t i = 0; i < N; ++i) {
+                const double a = (sc[order[i]] - mx) * scale - lnZ;
+                e[m].logp = a;
+                e[m].mass = (double)sizes[h * C + c] * exp(a);
+                e[m].h = h;
+                e[m].c = c;
+                e[m].pos = i;
+                total += e[m].mass;
+                ++m;
+            }
+        }
+    qsort(e, (size_t)E, sizeof(pool_entry), cmp_pool);
+    const double target = p * total;  /* total = sum over the pooled rows of |c| */
+    double cum = 0.0;
+    for (int64_t i = 0; i < E; ++i) {
+        cum += e[i].mass;
+        counts[e[i].h * C + e[i].c] += 1;
+        if (cum >= target) break;
+    }
+    free(order);
+    free(e);
+    return total > 0.0 ? cum / total : 1.0;
+}
+
 /* Selected keys of one cluster: the first n keys of the order, written in
  * ascending key index (R11). */
 void orc_emit(const double *s, int64_t N, int64_t n, int32_t *out)

@@ -357,3 +357,100 @@ def test_pipeline_tiny_config_invariants():
             assert (np.diff(lst) > 0).all()
         o = oracle.scope_attn_head(out["qr"], out["kr"], v[0, h].double().numpy(), out["q_labels"], out["lists"])
         assert np.isfinite(o).all()
+
+
+# ----------------------------------------------------------------------------- EG-Sparse (reading R17)
+def test_head_entropy_closed_forms():
+    N = 64
+    scale = 0.5
+    assert oracle.head_entropy(np.zeros((3, N)), [1, 2, 3], scale) == pytest.approx(1.0, abs=1e-12)  # uniform rows
+    # one key ahead by L: pi = (e^{aL}, 1, ..., 1) / (e^{aL} + N - 1), a two-valued distribution
+    L = 12.0
+    s = np.zeros((1, N))
+    s[0, 5] = L
+    z = np.exp(scale * L) + N - 1
+    p1, p0 = np.exp(scale * L) / z, 1.0 / z
+    H = -(p1 * np.log(p1) + (N - 1) * p0 * np.log(p0))
+    assert oracle.head_entropy(s, [7], scale) == pytest.approx(H / np.log(N), rel=1e-12)
+    # rows weigh by their query counts; an empty row weighs nothing
+    s2 = np.vstack([np.zeros(N), s[0], np.full(N, 3.0)])
+    e = oracle.head_entropy(s2, [3, 1, 0], scale)
+    assert e == pytest.approx((3 * 1.0 + 1 * H / np.log(N)) / 4, rel=1e-12)
+
+
+def test_head_entropy_matches_a_library_entropy():
+    from scipy.stats import entropy
+    rng = np.random.default_rng(11)
+    C, N, scale = 5, 40, 0.3
+    s = rng.standard_normal((C, N)) * 4
+    sizes = rng.integers(1, 9, C)
+    rows = [entropy(np.exp(scale * (r - r.max()))) for r in s]  # scipy normalises the weights itself
+    ref = float(np.dot(sizes, rows) / (sizes.sum() * np.log(N)))
+    assert oracle.head_entropy(s, sizes, scale) == pytest.approx(ref, rel=1e-12)
+
+
+def test_pooled_topp_hand_examples():
+    with open(os.path.join(os.path.dirname(__file__), "golden", "eg_pooled.json")) as f:
+        cases = json.load(f)["cases"]
+    for cs in cases:
+        sizes = np.array(cs["sizes"])
+        s = np.zeros(sizes.shape + (cs["N"],))  # equal scores: pi = 1/N everywhere
+        assert oracle.pooled_topp(s, sizes, cs["p"], 1.0).tolist() == cs["counts"], cs["work"]
+
+
+def test_pooled_topp_of_one_row_is_its_topp():
+    rng = np.random.default_rng(12)
+    for p in (0.3, 0.8, 0.9, 0.999):
+        s = rng.standard_normal(50) * 6
+        got = oracle.pooled_topp(s[None, None, :], np.array([[4]]), p, 0.4)
+        assert got[0, 0] == oracle.topp_count(s, p, 0.4)
+
+
+def test_pooled_topp_against_a_library_sort():
+    """An independent restatement of the pooled prefix (numpy lexsort over all
+    entries) on random tiny pools, with rows of unequal sizes and tied scores."""
+    rng = np.random.default_rng(13)
+    for trial in range(20):
+        Hp, C, N = 2, 3, 6
+        s = rng.integers(-3, 4, (Hp, C, N)).astype(np.float64)  # integer scores: many ties
+        sizes = rng.integers(1, 5, (Hp, C))
+        p, scale = rng.uniform(0.2, 0.95), 0.7
+        logp, mass, hs, cs, pos = [], [], [], [], []
+        for h in range(Hp):
+            for c in range(C):
+                row = s[h, c]
+                order = np.lexsort((np.arange(N), -row))  # score desc, index asc
+                a = (row[order] - row.max()) * scale
+                a -= np.log(np.exp(a).sum())
+                logp += list(a)
+                mass += list(sizes[h, c] * np.exp(a))
+                hs += [h] * N
+                cs += [c] * N
+                pos += list(range(N))
+        rank = np.lexsort((pos, cs, hs, -np.array(logp)))
+        cum = np.cumsum(np.array(mass)[rank])
+        m = int(np.searchsorted(cum, p * cum[-1] * (1 - 1e-15))) + 1  # first prefix reaching p
+        ref = np.zeros((Hp, C), np.int64)
+        for i in rank[:m]:
+            ref[hs[i], cs[i]] += 1
+        got, frac = oracle.pooled_topp(s, sizes, p, scale, with_mass=True)
+        assert (got == ref).all(), (trial, got, ref)
+        assert frac >= p * (1 - 1e-12)
+
+
+def test_eg_route_and_tau_zero_keeps_per_row_selection():
+    assert oracle.eg_route([0.1, 0.9, 0.2, 0.3, 0.95], 0.5, 2) == [[0], [2, 3], []]
+    assert oracle.eg_route([0.1, 0.2], 0.0, 2) == [[]]
+    rng = np.random.default_rng(14)
+    H, C, N = 3, 4, 30
+    scores = [rng.standard_normal((C, N)) * 5 for _ in range(H)]
+    sizes = [rng.integers(0, 6, C) for _ in range(H)]
+    _, pools, counts = oracle.eg_counts(scores, sizes, 0.9, 0.0, 2, 0.3)
+    assert all(not p for p in pools)
+    for h in range(H):
+        for c in range(C):
+            assert counts[h, c] == oracle.topp_count(scores[h][c], 0.9, 0.3)
+    # every head low-entropy, one group: the counts are one pool's
+    _, pools, counts = oracle.eg_counts(scores, sizes, 0.9, 1.01, H, 0.3)
+    assert pools == [list(range(H))]
+    assert (counts == oracle.pooled_topp(np.stack(scores), np.stack(sizes), 0.9, 0.3)).all()
