@@ -80,6 +80,12 @@ def lib():
         L.orc_head_entropy.restype = ctypes.c_double
         L.orc_pooled_topp.argtypes = [_d, _i64, _I, _I, _I, ctypes.c_double, ctypes.c_double, _i64]
         L.orc_pooled_topp.restype = ctypes.c_double
+        L.orc_block_ids.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int, ctypes.c_int32,
+                                    ctypes.c_int32, ctypes.c_int32, _i32]
+        L.orc_block_ids.restype = ctypes.c_int64
+        L.orc_block_select.argtypes = [_d, _i64, _I, ctypes.c_double, ctypes.c_double,
+                                       np.ctypeslib.ndpointer(dtype=np.int8, flags="C_CONTIGUOUS")]
+        L.orc_block_select.restype = ctypes.c_int64
         _lib = L
     return _lib
 
@@ -251,6 +257,55 @@ def eg_counts(scores_heads, sizes_heads, p: float, tau: float, group: int, scale
             counts[pool] = pooled_topp(np.stack([scores_heads[h] for h in pool]),
                                        np.stack([sizes_heads[h] for h in pool]), p, scale)
     return ent, pools, counts
+
+
+def block_ids(grid, kind: int, block):
+    """VMoBA block partition (R18): block id of every token and the block count."""
+    T, Hh, W = grid
+    ids = np.empty(T * Hh * W, np.int32)
+    nb = lib().orc_block_ids(T, Hh, W, int(kind), *[int(x) for x in block], ids)
+    return ids, int(nb)
+
+
+def block_means(x, ids, nb: int) -> np.ndarray:
+    """Mean row of every block (fp64); an empty block has a zero mean."""
+    x = _f64(x)
+    out = np.zeros((nb, x.shape[1]))
+    cnt = np.bincount(ids, minlength=nb).astype(np.float64)
+    np.add.at(out, ids, x)
+    return out / np.maximum(cnt, 1.0)[:, None]
+
+
+def block_select(s, sizes, p: float, scale: float):
+    """VMoBA threshold selection of one query cluster over blocks (R18):
+    (kept block flags, kept key count)."""
+    s = _f64(s)
+    keep = np.empty(s.shape[0], np.int8)
+    n = lib().orc_block_select(s, np.ascontiguousarray(sizes, np.int64), s.shape[0], float(p), float(scale), keep)
+    return keep.astype(bool), int(n)
+
+
+def vmoba_plan_head(q, k, p: "Params", kind: int, block, store_bf16: bool = False) -> dict:
+    """Block-granular variant for one head: SCOPE's RoPE and query k-means,
+    key blocks of the given partition scored by their mean key, threshold
+    selection of whole blocks; lists = the kept blocks' keys, ascending."""
+    q, k = _f64(q), _f64(k)
+    N, D = q.shape
+    scale = 1.0 / np.sqrt(D)
+    qr = rope3d(q, p.grid, p.d_split, p.theta)
+    kr = rope3d(k, p.grid, p.d_split, p.theta)
+    if store_bf16:
+        qr, kr = _round_bf16(qr), _round_bf16(kr)
+    qlab, qcent, qsizes = kmeans(qr, p.c_q, p.iters, p.seed)
+    ids, nb = block_ids(p.grid, kind, block)
+    kbar = block_means(kr, ids, nb)
+    bsizes = np.bincount(ids, minlength=nb).astype(np.int64)
+    lists, n = [], np.zeros(p.c_q, np.int64)
+    for c in range(p.c_q):
+        keep, n[c] = block_select(qcent[c] @ kbar.T, bsizes, p.top_p, scale)
+        lists.append(np.nonzero(keep[ids])[0].astype(np.int32))
+    return dict(qr=qr, kr=kr, q_labels=qlab, q_centroids=qcent, q_sizes=qsizes, block_ids=ids,
+                block_means=kbar, n=n, lists=lists)
 
 
 def attention_rows(q_rows, K, V, sel, scale: float) -> np.ndarray:

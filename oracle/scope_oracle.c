@@ -384,6 +384,68 @@ double orc_pooled_topp(const double *s, const int64_t *sizes, int64_t Hp, int64_
     return total > 0.0 ? cum / total : 1.0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* VMoBA block-granular selection ["VMoBA: Mixture-of-Block Attention for    */
+/* Video Diffusion Models", abstract items (1) a layer-wise recurrent 1D-2D- */
+/* 3D block partition and (3) threshold selection of blocks by cumulative    */
+/* similarity].  Readings (R18):                                           */
+/*  - kind 1: runs of bt*bh*bw consecutive tokens in raster order; kind 2:  */
+/*    bh x bw tiles inside each frame; kind 3: bt x bh x bw cubes; ragged   */
+/*    edge blocks; blocks numbered in raster order of their corners.  The   */
+/*    caller cycles the kind with the layer index (the recurrent scheme).   */
+/*  - a key block's representative is the mean of its post-RoPE keys; query */
+/*    cluster c scores block b by s_c(b) = qbar_c . kbar_b;                  */
+/*  - blocks are ranked by s_c(b) descending; each weighs |b| e^{scale s};   */
+/*    the shortest prefix whose weight reaches p of the total is kept, and  */
+/*    blocks tied with the last kept one are kept too (whole blocks only).  */
+/* ------------------------------------------------------------------------ */
+
+/* Block id of every token of a T x Hh x W grid; returns the block count. */
+int64_t orc_block_ids(int32_t T, int32_t Hh, int32_t W, int kind, int32_t bt, int32_t bh, int32_t bw,
+                      int32_t *ids)
+{
+    const int64_t N = (int64_t)T * Hh * W;
+    if (kind == 1) {
+        const int64_t len = (int64_t)bt * bh * bw;
+        for (int64_t n = 0; n < N; ++n) ids[n] = (int32_t)(n / len);
+        return (N + len - 1) / len;
+    }
+    const int64_t nbt = kind == 2 ? T : (T + bt - 1) / bt;
+    const int64_t nbh = (Hh + bh - 1) / bh, nbw = (W + bw - 1) / bw;
+    for (int64_t n = 0; n < N; ++n) {
+        const int64_t t = n / ((int64_t)Hh * W), y = (n / W) % Hh, x = n % W;
+        const int64_t tb = kind == 2 ? t : t / bt;
+        ids[n] = (int32_t)((tb * nbh + y / bh) * nbw + x / bw);
+    }
+    return nbt * nbh * nbw;
+}
+
+/* Keys kept by one query cluster: s [Nb] block scores, sizes [Nb]; keep[b]
+ * set to 1 for kept blocks; returns the kept key count. */
+int64_t orc_block_select(const double *s, const int64_t *sizes, int64_t Nb, double p, double scale, int8_t *keep)
+{
+    int64_t *order = (int64_t *)malloc((size_t)(Nb > 0 ? Nb : 1) * sizeof(int64_t));
+    orc_order(s, Nb, order);
+    double mx = -INFINITY, total = 0.0;
+    for (int64_t b = 0; b < Nb; ++b)
+        if (sizes[b] > 0 && s[b] > mx) mx = s[b];
+    for (int64_t b = 0; b < Nb; ++b) total += (double)sizes[b] * exp((s[b] - mx) * scale);
+    for (int64_t b = 0; b < Nb; ++b) keep[b] = 0;
+    int64_t kept = 0;
+    double cum = 0.0, cut = INFINITY;
+    for (int64_t i = 0; i < Nb; ++i) {
+        const int64_t b = order[i];
+        if (sizes[b] <= 0) continue;
+        if (cum >= p * total && s[b] < cut) break;  /* reached, and past the last kept score */
+        keep[b] = 1;
+        kept += sizes[b];
+        cum += (double)sizes[b] * exp((s[b] - mx) * scale);
+        if (cum >= p * total && cut == INFINITY) cut = s[b];
+    }
+    free(order);
+    return kept;
+}
+
 /* Selected keys of one cluster: the first n keys of the order, written in
  * ascending key index (R11). */
 void orc_emit(const double *s, int64_t N, int64_t n, int32_t *out)

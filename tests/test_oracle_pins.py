@@ -454,3 +454,69 @@ def test_eg_route_and_tau_zero_keeps_per_row_selection():
     _, pools, counts = oracle.eg_counts(scores, sizes, 0.9, 1.01, H, 0.3)
     assert pools == [list(range(H))]
     assert (counts == oracle.pooled_topp(np.stack(scores), np.stack(sizes), 0.9, 0.3)).all()
+
+
+# ----------------------------------------------------------------------------- VMoBA blocks (reading R18)
+@pytest.mark.parametrize("grid", [(3, 7, 8), (5, 4, 9), (1, 1, 13)])
+@pytest.mark.parametrize("kind,block", [(1, (2, 2, 3)), (2, (1, 3, 4)), (3, (2, 3, 4)), (3, (1, 1, 1))])
+def test_block_partition_geometry(grid, kind, block):
+    T, Hh, W = grid
+    N = T * Hh * W
+    ids, nb = oracle.block_ids(grid, kind, block)
+    assert ids.min() == 0 and ids.max() == nb - 1 and len(np.unique(ids)) == nb  # every block used
+    n = np.arange(N)
+    t, y, x = n // (Hh * W), (n // W) % Hh, n % W
+    bt, bh, bw = block
+    for b in range(nb):
+        mem = np.nonzero(ids == b)[0]
+        if kind == 1:  # runs of consecutive tokens
+            assert (np.diff(mem) == 1).all() and len(mem) <= bt * bh * bw
+        else:
+            span_t = np.ptp(t[mem]) + 1
+            assert span_t <= (1 if kind == 2 else bt)
+            assert np.ptp(y[mem]) + 1 <= bh and np.ptp(x[mem]) + 1 <= bw
+    sizes = np.bincount(ids)
+    if kind == 1:
+        assert nb == -(-N // (bt * bh * bw))
+        assert (sizes[:-1] == bt * bh * bw).all()
+    else:
+        ct = T if kind == 2 else -(-T // bt)
+        assert nb == ct * -(-Hh // bh) * -(-W // bw)
+        assert sizes.max() == (1 if kind == 2 else min(bt, T)) * min(bh, Hh) * min(bw, W)
+
+
+def test_block_mean_scores_are_member_averages():
+    rng = np.random.default_rng(21)
+    k = rng.standard_normal((3 * 7 * 8, 16))
+    q = rng.standard_normal(16)
+    ids, nb = oracle.block_ids((3, 7, 8), 3, (2, 3, 4))
+    kbar = oracle.block_means(k, ids, nb)
+    for b in range(nb):
+        mem = ids == b
+        assert q @ kbar[b] * mem.sum() == pytest.approx((k[mem] @ q).sum(), rel=1e-12, abs=1e-12)
+
+
+def test_block_select_hand_examples():
+    with open(os.path.join(os.path.dirname(__file__), "golden", "vmoba_blocks.json")) as f:
+        cases = json.load(f)["cases"]
+    for cs in cases:
+        keep, n = oracle.block_select(np.array(cs["scores"]), np.array(cs["sizes"]), cs["p"], 1.0)
+        assert keep.tolist() == cs["keep"] and n == cs["kept_keys"], cs["work"]
+
+
+def test_single_token_blocks_reduce_to_per_key_topp():
+    rng = np.random.default_rng(22)
+    for p in (0.5, 0.9, 0.97):
+        s = rng.standard_normal(200) * 5  # continuous scores: no ties
+        keep, n = oracle.block_select(s, np.ones(200, np.int64), p, 0.3)
+        m = oracle.topp_count(s, p, 0.3)
+        assert n == m
+        assert (np.nonzero(keep)[0] == oracle.emit(s, m)).all()
+
+
+def test_block_select_grows_with_p():
+    rng = np.random.default_rng(23)
+    s = rng.standard_normal(60) * 3
+    sizes = rng.integers(1, 20, 60)
+    counts = [oracle.block_select(s, sizes, p, 0.5)[1] for p in np.linspace(0.05, 1.0, 40)]
+    assert all(a <= b for a, b in zip(counts, counts[1:])) and counts[-1] == sizes.sum()
