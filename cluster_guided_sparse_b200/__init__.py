@@ -26,7 +26,7 @@ SCOPE_F32, SCOPE_BF16, SCOPE_I32, SCOPE_I64 = 0, 1, 2, 3
 STATUS = {0: "SCOPE_OK", 1: "SCOPE_EINVAL", 2: "SCOPE_ESHAPE", 3: "SCOPE_EDTYPE", 4: "SCOPE_EALIGN",
           5: "SCOPE_EWORKSPACE", 6: "SCOPE_ECAPACITY", 7: "SCOPE_ECUDA", 8: "SCOPE_ETIMEOUT", 9: "SCOPE_EDEVICE"}
 VIEWS = ["qr", "kr", "q_labels", "q_centroids", "q_sizes", "q_perm", "q_start", "k_codes", "k_cent_t",
-         "k_cent_h", "k_cent_w", "lut", "r", "kh", "n", "offsets", "indices", "error"]
+         "k_cent_h", "k_cent_w", "lut", "r", "kh", "n", "offsets", "indices", "error", "eg_entropy", "eg_pool"]
 _TORCH_DT = {SCOPE_F32: torch.float32, SCOPE_BF16: torch.bfloat16, SCOPE_I32: torch.int32, SCOPE_I64: torch.int64}
 
 
@@ -45,7 +45,9 @@ class ScopeParams(ctypes.Structure):
                 ("c_h", ctypes.c_int32), ("c_w", ctypes.c_int32), ("iters", ctypes.c_int32),
                 ("init_seed", ctypes.c_uint32), ("top_p", ctypes.c_float), ("k_min", ctypes.c_int32),
                 ("online_topk", ctypes.c_int32), ("fixed_cluster_size", ctypes.c_int32),
-                ("compensate", ctypes.c_int32)]
+                ("compensate", ctypes.c_int32), ("eg_tau", ctypes.c_float), ("eg_group", ctypes.c_int32),
+                ("block_kind", ctypes.c_int32), ("block_t", ctypes.c_int32), ("block_h", ctypes.c_int32),
+                ("block_w", ctypes.c_int32)]
 
 
 class ScopeView(ctypes.Structure):
@@ -133,7 +135,8 @@ def make_params(w=None, **kw):
         f = dict(d_t=w.d_split[0], d_h=w.d_split[1], d_w=w.d_split[2], theta=w.theta, c_q=w.c_q,
                  c_t=w.c_sub[0], c_h=w.c_sub[1], c_w=w.c_sub[2], iters=w.iters, init_seed=0, top_p=w.top_p,
                  k_min=w.k_min, online_topk=w.online_topk, fixed_cluster_size=w.fixed_cluster_size,
-                 compensate=w.compensate)
+                 compensate=w.compensate, eg_tau=w.eg_tau, eg_group=w.eg_group, block_kind=w.block_kind,
+                 block_t=w.block_dims[0], block_h=w.block_dims[1], block_w=w.block_dims[2])
         grid = tuple(w.grid)
     else:
         grid = (0, 0, 0)

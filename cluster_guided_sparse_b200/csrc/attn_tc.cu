@@ -409,7 +409,15 @@ __global__ void __launch_bounds__(1024) tc_items_kernel(const int32_t *sizes, in
 
 }  // namespace tc
 
-constexpr size_t tc_smem_bytes(int D) { return (size_t)(2 * tc::BM * D * 2 + 4 * tc::BN * D * 2) + 1024; }
+// Dynamic shared memory per CTA.  Every CTA allocates all 512 TMEM columns,
+// so a second CTA on the same SM would only wait inside tcgen05.alloc: the
+// D = 64 tiles (97 KB) are padded past half of the SM's 228 KB so that the
+// scheduler places one CTA per SM, as for D = 128.
+constexpr size_t tc_smem_bytes(int D)
+{
+    const size_t need = (size_t)(2 * tc::BM * D * 2 + 4 * tc::BN * D * 2) + 1024;
+    return need > 120 * 1024 ? need : 120 * 1024;
+}
 
 cudaError_t attn_tc_configure()
 {

@@ -12,6 +12,7 @@ constexpr int kMaxClusters = 1024;
 constexpr int kTQ = 128;        // query rows per attention tile
 constexpr int kMaxItems = 65536; // c_t * c_h * c_w bound (distinct code triples)
 constexpr int kScanTileCounters = 4096;  // block counters per tile of the label-sort scan
+constexpr int kMaxBlocks = 16384;        // key blocks of the VMoBA block mode
 
 // Device error word bits (workspace int32[4]).
 constexpr int kErrRange = 1;

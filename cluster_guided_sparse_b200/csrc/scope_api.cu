@@ -51,8 +51,13 @@ void run_selection(const float *lut, const int32_t *codes, const int32_t *item_i
                    const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch, int Cw,
                    int BH, float top_p,
                    float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes, int32_t *r, int32_t *n,
-                   int32_t *kh, long long *offsets, int32_t *indices, int online, void *state, cudaStream_t st);
+                   int32_t *kh, long long *offsets, int32_t *indices, int online, void *state, int B, float eg_tau,
+                   int eg_group, void *eg_state, int whole_items, cudaStream_t st);
 size_t selection_state_bytes(int64_t clusters);
+size_t eg_state_bytes(int64_t B, int64_t H, int64_t Cq, int group);
+int block_count(int T, int Hh, int W, int kind, int bt, int bh, int bw);
+void launch_blocks(int T, int Hh, int W, int kind, int bt, int bh, int bw, const __nv_bfloat16 *kr, int32_t *codes,
+                   float *cent, float *cn, int32_t *sizes, int BH, int N, int D, cudaStream_t st);
 }  // namespace scope
 
 using namespace scope;
@@ -90,9 +95,9 @@ struct Layout {
     int64_t cap;
     size_t qr, kr, qnorm, tab, stats, maxabs, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist, q_tsum;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3], k_tsum[3];
-    size_t sel_state, lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
+    size_t sel_state, eg_state, lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
     size_t bis_order, bis_delta, bis_aux, q_chi, q_clo, q_sums, k_sums[3], sums_bytes, lse, vmean;
-    bool comp;
+    bool comp, eg, blocks;
     size_t total;
 };
 
@@ -234,6 +239,28 @@ scope_status check_params(const scope_tensor *q, const scope_grid *g, const scop
     }
     if (p->fixed_cluster_size < 0) return fail(SCOPE_EINVAL, "params: fixed_cluster_size must be >= 0");
     if (p->compensate != 0 && p->compensate != 1) return fail(SCOPE_EINVAL, "params: compensate must be 0 or 1");
+    if (!(p->eg_tau >= 0.f && p->eg_tau <= 2.f))
+        return fail(SCOPE_EINVAL, "params: eg_tau must be in [0, 2] (0 = no EG-Sparse routing)");
+    if (p->eg_tau > 0.f && (p->eg_group < 1 || p->eg_group > 64))
+        return fail(SCOPE_EINVAL, "params: eg_group must be in [1, 64] when eg_tau > 0");
+    if (p->eg_tau > 0.f && (int64_t)(p->eg_group < q->H ? p->eg_group : q->H) * q->N > ((int64_t)1 << 24))
+        return fail(SCOPE_EINVAL, "params: a pool's queries (min(eg_group, H) * N) must be <= 2^24");
+    if (p->block_kind < 0 || p->block_kind > 3) return fail(SCOPE_EINVAL, "params: block_kind must be 0..3");
+    if (p->block_kind > 0) {
+        if (!has_grid) return fail(SCOPE_EINVAL, "block_kind needs a grid");
+        if (p->block_t < 1 || p->block_h < 1 || p->block_w < 1)
+            return fail(SCOPE_EINVAL, "params: block_t, block_h, block_w must be >= 1");
+        if (p->k_min != 0 || p->online_topk != 0 || p->eg_tau > 0.f || p->fixed_cluster_size > 0 || p->compensate)
+            return fail(SCOPE_EINVAL, "block_kind needs k_min = 0, online_topk = 0, eg_tau = 0, no "
+                                      "fixed_cluster_size and no compensate");
+        if ((int64_t)p->block_t * p->block_h * p->block_w > N)
+            return fail(SCOPE_EINVAL, "params: a block must not exceed N tokens");
+        const int nb = block_count(g->T, g->Hh, g->W, p->block_kind, p->block_t, p->block_h, p->block_w);
+        if (nb > kMaxBlocks) return fail(SCOPE_EINVAL, "block_kind: %d blocks > %d", nb, kMaxBlocks);
+        if (p->c_q < 1 || p->c_q > N || p->c_q > kMaxClusters)
+            return fail(SCOPE_EINVAL, "params: c_q must be in [1, min(N, %d)]", kMaxClusters);
+        return SCOPE_OK;
+    }
     if (p->compensate && p->fixed_cluster_size == 0)
         return fail(SCOPE_EINVAL, "params: compensate needs the ClusterAttention variant (fixed_cluster_size > 0)");
     if (p->fixed_cluster_size > 0) {
@@ -270,16 +297,24 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.f32 = q->dtype == SCOPE_F32;
     L.bisect = p->fixed_cluster_size > 0;
     const int ds[3] = {p->d_t, p->d_h, p->d_w};
+    L.blocks = p->block_kind > 0;
     if (L.bisect) {
         const int Cn = (int)(L.N / p->fixed_cluster_size);
         L.Cq = Cn;
         L.C[0] = Cn; L.C[1] = 1; L.C[2] = 1;
+    } else if (L.blocks) {
+        L.Cq = p->c_q;
+        L.C[0] = block_count(g->T, g->Hh, g->W, p->block_kind, p->block_t, p->block_h, p->block_w);
+        L.C[1] = 1; L.C[2] = 1;
     } else {
         L.Cq = p->c_q;
         L.C[0] = p->c_t; L.C[1] = p->c_h; L.C[2] = p->c_w;
     }
     for (int s = 0; s < 3; ++s) L.ds[s] = ds[s];
-    L.off[0] = 0; L.off[1] = ds[0]; L.off[2] = ds[0] + ds[1];
+    if (L.blocks) {  // one "subspace": the whole rotated key, one centroid per block
+        L.ds[0] = (int)L.D; L.ds[1] = 0; L.ds[2] = 0;
+    }
+    L.off[0] = 0; L.off[1] = L.ds[0]; L.off[2] = L.ds[0] + L.ds[1];
     L.Csum = L.C[0] + L.C[1] + L.C[2];
     L.P = L.C[0] * L.C[1] * L.C[2];
     L.Pcap = (int)(L.P < L.N ? L.P : L.N);
@@ -326,7 +361,7 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.vmean = take(cur, L.comp ? BH * L.C[0] * D * 4 : 0);
     L.k_codes = take(cur, 3 * BH * N * 4);
     for (int s = 0; s < 3; ++s) {
-        L.k_cent[s] = take(cur, BH * L.C[s] * (ds[s] > 0 ? ds[s] : 1) * 4);
+        L.k_cent[s] = take(cur, BH * L.C[s] * (L.ds[s] > 0 ? L.ds[s] : 1) * 4);
         L.k_cn[s] = take(cur, BH * L.C[s] * 4);
         L.k_sizes[s] = take(cur, BH * L.C[s] * 4);
         L.k_perm[s] = take(cur, BH * N * 4);
@@ -336,6 +371,8 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     }
     L.lut = take(cur, BH * L.Cq * L.Csum * 4);
     L.sel_state = take(cur, selection_state_bytes(BH * L.Cq));
+    L.eg = p->eg_tau > 0.f;
+    L.eg_state = take(cur, L.eg ? eg_state_bytes(L.B, L.H, L.Cq, p->eg_group) : 0);
     L.item_hist = take(cur, BH * L.P * 4);
     L.item_id = take(cur, BH * L.Pcap * 4);
     L.item_cnt = take(cur, BH * L.Pcap * 4);
@@ -516,12 +553,21 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     KmBatch qonly{};
     qonly.p[0] = all.p[3];
     qonly.count = 1;
+    if (L.blocks) {
+        // VMoBA block mode: only the queries are clustered; the keys' codes and
+        // centroids come from the block partition
+        all = qonly;
+        keys.count = 0;
+        launch_blocks(grid->T, grid->Hh, grid->W, p->block_kind, p->block_t, p->block_h, p->block_w,
+                      at<__nv_bfloat16>(ws, L.kr), at<int32_t>(ws, L.k_codes), at<float>(ws, L.k_cent[0]),
+                      at<float>(ws, L.k_cn[0]), at<int32_t>(ws, L.k_sizes[0]), BH, N, D, s);
+    }
     int32_t *fix_count = at<int32_t>(ws, L.fix);
     int32_t *fix_list = fix_count + 4;
     bool tc_ok = true;
     auto assign = [&]() {
         if (tc_q) {
-            launch_km_assign_direct(keys, BH, N, D, s);
+            if (keys.count) launch_km_assign_direct(keys, BH, N, D, s);
             tc_ok = tc_ok && launch_km_assign_tc(all.p[3], at<__nv_bfloat16>(ws, L.q_chi),
                                                  at<__nv_bfloat16>(ws, L.q_clo), BH, N, D, at<float>(ws, L.qnorm),
                                                  fix_list, fix_count, at<int32_t>(ws, L.stats) + 4, s);
@@ -553,7 +599,8 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
                   L.Cq, L.C[0], L.C[1], L.C[2], BH, p->top_p, 1.0f / sqrtf((float)D), p->k_min,
                   at<int32_t>(ws, L.stats) + 4,
                   at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.r), at<int32_t>(ws, L.n), at<int32_t>(ws, L.kh),
-                  at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, ws + L.sel_state, s);
+                  at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, ws + L.sel_state, (int)L.B,
+                  p->eg_tau, p->eg_group, L.eg ? ws + L.eg_state : nullptr, L.blocks ? 1 : 0, s);
     if ((st = launch_status("selection")) != SCOPE_OK) return st;
 
     scope_plan_s *h = (scope_plan_s *)malloc(sizeof(scope_plan_s));
@@ -741,6 +788,14 @@ extern "C" scope_status scope_plan_view(const scope_plan_t *plan, int which, sco
     case SCOPE_VIEW_OFFSETS: set(L.offsets, SCOPE_I64, 1, L.BH * L.Cq + 1, 0, 0, 0); break;
     case SCOPE_VIEW_INDICES: set(L.indices, SCOPE_I32, 1, L.cap, 0, 0, 0); break;
     case SCOPE_VIEW_ERROR: set(L.stats + 16, SCOPE_I32, 1, 4, 0, 0, 0); break;
+    case SCOPE_VIEW_EG_ENTROPY:
+        if (!L.eg) return fail(SCOPE_EINVAL, "no EG-Sparse routing in this plan (eg_tau = 0)");
+        set(L.eg_state, SCOPE_F32, 2, B, H, 0, 0);
+        break;
+    case SCOPE_VIEW_EG_POOL:
+        if (!L.eg) return fail(SCOPE_EINVAL, "no EG-Sparse routing in this plan (eg_tau = 0)");
+        set(L.eg_state + L.BH * 4, SCOPE_I32, 2, B, H, 0, 0);
+        break;
     default: return fail(SCOPE_EINVAL, "view id %d out of range", which);
     }
     *out = v;

@@ -33,6 +33,7 @@ struct SelArgs {
     int Pcap, N, Cq, Ct, Ch, Cw, BH;
     float top_p, inv_sqrt_d;
     int k_min;
+    int whole_items;          // block mode: the cut takes every key tied at the cut score
     int32_t *err;             // device error word
 };
 
@@ -140,6 +141,7 @@ struct SelShared {
     unsigned long long utmp[33];
     int itmp[33];
     float fmin[32], fmax[32];
+    double dz[32], da[32];
     uint32_t prefix;
     int coarse;  // the coarse bucket being refined (-1: none)
     unsigned long long above_met, run_met, bucket_met, new_above_met;
@@ -185,8 +187,10 @@ struct ClusterCut {
     float smin, smax;
     uint32_t key;     // order key of the last key the Top-p prefix takes
     int32_t need;     // keys it takes at that key
-    int32_t taken;    // the Top-p count |P_c|
-    int32_t pad[3];
+    int32_t taken;    // the Top-p count |P_c| (-1: set by a pooled selection)
+    float ent;        // entropy (nats) of the row's proxy softmax
+    float lnz;        // ln of its normaliser sum_j e^{(s_j - smax) / sqrt(D)}
+    int32_t pad;
 };
 
 // The order key of item i (cached, or recomputed from the table row).
@@ -282,7 +286,7 @@ __device__ bool refine_pass(SelShared &S, const ItemKeys &K, const int32_t *cnts
 // which exact integer metrics rule out).
 __device__ int refine(SelShared &S, const ItemKeys &K, const int32_t *cnts, int n_items, const CoarseMap &cm,
                       float smax, float inv_sqrt_d, bool by_mass, unsigned long long target, uint32_t *cut_key,
-                      int *need_at_cut)
+                      int *need_at_cut, bool whole = false)
 {
     if (threadIdx.x == 0) S.prefix = 0u;
     __syncthreads();
@@ -292,7 +296,7 @@ __device__ int refine(SelShared &S, const ItemKeys &K, const int32_t *cnts, int 
     // every key in the final bucket has the same score, hence the same metric
     const unsigned long long per = S.bucket_met / (unsigned long long)S.bucket_cnt;
     const unsigned long long rest = target - S.above_met;
-    const int need = (int)((rest + per - 1) / per);
+    const int need = whole ? S.bucket_cnt : (int)((rest + per - 1) / per);
     *cut_key = S.prefix;
     *need_at_cut = need;
     return S.above_cnt + need;
@@ -362,6 +366,7 @@ __global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r
     __syncthreads();
     const bool sel = a.top_p < 1.0f;
     unsigned long long wsum = 0ull;
+    double zs = 0.0, as = 0.0;  // sum cnt e^x and sum cnt e^x x, x = (s - smax) / sqrt(D): the row entropy
     for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
         const float sc = key_score(K(i));
         const int b = cm(sc);
@@ -370,7 +375,19 @@ __global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r
             const unsigned long long w = (unsigned long long)cnts[i] * item_mass(sc, smax, a.inv_sqrt_d);
             atomicAdd(&S.met[b], w);
             wsum += w;
+            const float x = (sc - smax) * a.inv_sqrt_d;
+            const double e = (double)cnts[i] * (double)expf(x);
+            zs += e;
+            as += e * (double)x;
         }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        zs += __shfl_xor_sync(0xffffffffu, zs, o);
+        as += __shfl_xor_sync(0xffffffffu, as, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        S.dz[threadIdx.x >> 5] = zs;
+        S.da[threadIdx.x >> 5] = as;
     }
     __syncthreads();
     int32_t *hist_out = coarse_hist + bhc * kBuckets;
@@ -389,7 +406,9 @@ __global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r
         pick_bucket(S, kBuckets, target);
         if (threadIdx.x == 0) S.coarse = S.bucket;
         __syncthreads();
-        m = S.coarse >= 0 ? refine(S, K, cnts, n_items, cm, smax, a.inv_sqrt_d, true, target, &key, &need) : -1;
+        m = S.coarse >= 0 ? refine(S, K, cnts, n_items, cm, smax, a.inv_sqrt_d, true, target, &key, &need,
+                                   a.whole_items != 0)
+                          : -1;
         if (m < 0) {
             if (threadIdx.x == 0) set_error(a.err, kErrRange, 0x100 + c);
             m = a.N;
@@ -405,8 +424,285 @@ __global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r
         cut.key = key;
         cut.need = need;
         cut.taken = sel ? m : a.N;
-        cut.pad[0] = cut.pad[1] = cut.pad[2] = 0;
+        double Z = 0.0, A = 0.0;  // fixed combination order: deterministic
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            Z += S.dz[w];
+            A += S.da[w];
+        }
+        cut.lnz = sel && Z > 0.0 ? (float)log(Z) : 0.f;
+        cut.ent = sel && Z > 0.0 ? (float)(log(Z) - A / Z) : 0.f;
+        cut.pad = 0;
         cuts[bhc] = cut;
+    }
+}
+
+// -------------------------------------------------------------- EG-Sparse
+// "EG-Sparse" (abstract): low-entropy heads are routed to a grouped
+// cross-head pool, high-entropy heads keep per-row selection, using only
+// scores the sparse pipeline already has.  Reading: a head's entropy is the
+// query-weighted mean of its rows' proxy-softmax entropies over ln N; heads
+// below eg_tau are grouped eg_group at a time (per batch entry) and a group's
+// low-entropy heads form one pool, in which every (head, cluster, key) entry
+// competes by ln pi = (s - smax) / sqrt(D) - ln Z of its row and carries mass
+// |c| pi; the shortest prefix reaching top_p of the pool's mass is kept (ties:
+// head, then cluster, then the row's own key order), and a row's Top-p count
+// is its number of kept entries.  Clusters without queries stay out of the
+// pool and keep their own count.
+//
+// The pooled select mirrors the per-row one across CTAs: coarse buckets of
+// ln pi over [-kLambdaSpan, 0] (entries below share bucket 0), then a radix
+// refine on the exact fp32 order key of ln pi, each pass a histogram that the
+// clusters' CTAs add into the pool's buffer and one CTA per pool reads.  Pool
+// masses are 64-bit fixed point in 2^-32 units (a pool of 64 heads of 2^24
+// queries stays below 2^63).
+constexpr float kLambdaSpan = 64.f;
+constexpr double kPoolMassScale = 4294967296.0;  // 2^32
+
+struct PoolSel {
+    unsigned long long met[kBuckets];  // histogram of the pass in progress
+    int cnt[kBuckets];
+    unsigned long long target;         // ceil(top_p * pool mass)
+    unsigned long long above_met;      // mass strictly above the chosen range
+    uint32_t prefix;                   // order-key bits fixed so far
+    int coarse;                        // chosen coarse bucket (-1: none)
+    int ok;
+    int pad;
+};
+
+__device__ __forceinline__ int lambda_bucket(float lam)
+{
+    const float t = __fmul_rn(__fadd_rn(lam, kLambdaSpan), (float)kBuckets / kLambdaSpan);
+    return t <= 0.f ? 0 : (t < (float)(kBuckets - 1) ? (int)t : kBuckets - 1);
+}
+
+// ln pi of an item of row (c, bh): the same fp32 operations in every pass
+__device__ __forceinline__ float item_lambda(float sc, const ClusterCut &cut, float inv_sqrt_d)
+{
+    return __fsub_rn((sc - cut.smax) * inv_sqrt_d, cut.lnz);
+}
+
+// Head entropies and routing, one CTA per batch entry, one warp per head.
+__global__ void __launch_bounds__(1024) eg_route_kernel(const ClusterCut *cuts, const int32_t *sizes, float *entropy,
+                                                        int32_t *pool, int H, int Cq, int N, float tau, int group)
+{
+    const int b = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ngroups = (H + group - 1) / group;
+    for (int h = warp; h < H; h += blockDim.x >> 5) {
+        const int64_t bh = (int64_t)b * H + h;
+        double num = 0.0, den = 0.0;
+        for (int c = lane; c < Cq; c += 32) {
+            const int z = sizes[bh * Cq + c];
+            num += (double)z * (double)cuts[bh * Cq + c].ent;
+            den += (double)z;
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            num += __shfl_xor_sync(0xffffffffu, num, o);
+            den += __shfl_xor_sync(0xffffffffu, den, o);
+        }
+        if (lane == 0) {
+            const float e = den > 0.0 && N > 1 ? (float)(num / (den * log((double)N))) : 0.f;
+            entropy[bh] = e;
+            pool[bh] = e < tau ? b * ngroups + h / group : -1;
+        }
+    }
+}
+
+// One pass over the items of one pooled cluster: the coarse histogram
+// (pass < 0) or the refine digit [shift, shift + width) among the chosen
+// range, added into the pool's histogram.
+__global__ void __launch_bounds__(kSelThreads) eg_hist_kernel(SelArgs a, const ClusterCut *cuts,
+                                                              const int32_t *sizes, const int32_t *pool,
+                                                              PoolSel *pools, int shift, int width)
+{
+    extern __shared__ __align__(16) float L[];
+    __shared__ unsigned long long hmet[kBuckets];
+    __shared__ int hcnt[kBuckets];
+    const int c = blockIdx.x, bh = blockIdx.y;
+    const int64_t bhc = (int64_t)bh * a.Cq + c;
+    const int pid = pool[bh];
+    const int sz = sizes[bhc];
+    if (pid < 0 || sz <= 0) return;
+    PoolSel &P = pools[pid];
+    const bool coarse = shift < 0;
+    if (!coarse && (P.coarse < 0 || !P.ok)) return;
+    const int Csum = a.Ct + a.Ch + a.Cw;
+    const float *lrow = a.lut + bhc * Csum;
+    for (int e = threadIdx.x; e < Csum; e += blockDim.x) L[e] = lrow[e];
+    const int nb = coarse ? kBuckets : 1 << width;
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        hmet[i] = 0ull;
+        hcnt[i] = 0;
+    }
+    __syncthreads();
+    const ClusterCut cut = cuts[bhc];
+    const int n_items = a.item_n[bh];
+    const int32_t *ids = a.item_id + (int64_t)bh * a.Pcap;
+    const int32_t *cnts = a.item_cnt + (int64_t)bh * a.Pcap;
+    const int hi = shift + width;
+    const uint32_t pre = P.prefix;
+    const int cb = P.coarse;
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const float lam = item_lambda(item_score(L, ids[i], a.Ch, a.Cw, a.Ct), cut, a.inv_sqrt_d);
+        const int lb = lambda_bucket(lam);
+        int d;
+        if (coarse) {
+            d = lb;
+        } else {
+            const uint32_t u = ordered_key(lam);
+            if (lb != cb || (hi < 32 && (u >> hi) != (pre >> hi))) continue;
+            d = (int)((u >> shift) & (uint32_t)(nb - 1));
+        }
+        const unsigned long long m =
+            (unsigned long long)sz * (unsigned long long)llrint((double)cnts[i] * (double)expf(lam) * kPoolMassScale);
+        atomicAdd(&hcnt[d], cnts[i]);
+        atomicAdd(&hmet[d], m);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb; i += blockDim.x)
+        if (hcnt[i]) {
+            atomicAdd(&P.cnt[i], hcnt[i]);
+            atomicAdd(&P.met[i], hmet[i]);
+        }
+}
+
+// One CTA per pool: reads the pass's histogram (and clears it for the next
+// pass), then picks the bucket where the pool's running mass reaches the
+// target; the coarse pass (shift < 0) first sets the target.
+__global__ void __launch_bounds__(kSelThreads) eg_pick_kernel(PoolSel *pools, float top_p, int shift, int width,
+                                                              int32_t *err)
+{
+    __shared__ SelShared S;
+    PoolSel &P = pools[blockIdx.x];
+    const bool coarse = shift < 0;
+    if (!coarse && (P.coarse < 0 || !P.ok)) return;
+    const int nb = coarse ? kBuckets : 1 << width;
+    unsigned long long w = 0ull;
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        S.met[i] = P.met[i];
+        S.cnt[i] = P.cnt[i];
+        w += S.met[i];
+        P.met[i] = 0ull;
+        P.cnt[i] = 0;
+    }
+    unsigned long long W;
+    block_excl_scan(w, S.utmp, W);
+    if (coarse) {
+        if (W == 0ull) {  // no pooled rows in this group
+            if (threadIdx.x == 0) {
+                P.coarse = -1;
+                P.ok = 1;
+            }
+            return;
+        }
+        unsigned long long t = (unsigned long long)ceil((double)top_p * (double)W);
+        t = t < 1ull ? 1ull : (t > W ? W : t);
+        if (threadIdx.x == 0) {
+            P.target = t;
+            P.above_met = 0ull;
+            P.prefix = 0u;
+        }
+    }
+    if (threadIdx.x == 0) {
+        S.above_met = P.above_met;
+        S.above_cnt = 0;
+    }
+    __syncthreads();
+    pick_bucket(S, nb, P.target);
+    if (threadIdx.x == 0) {
+        if (S.bucket < 0) {
+            P.ok = 0;
+            P.coarse = -1;
+            set_error(err, kErrRange, 0x400 + (int)blockIdx.x);
+        } else {
+            P.ok = 1;
+            P.above_met = S.above_met;
+            if (coarse) P.coarse = S.bucket;
+            else P.prefix |= (uint32_t)S.bucket << shift;
+        }
+    }
+}
+
+// Keys of every pooled cluster above and at the pool's cut (order key of ln pi).
+__global__ void __launch_bounds__(kSelThreads) eg_count_kernel(SelArgs a, const ClusterCut *cuts,
+                                                               const int32_t *sizes, const int32_t *pool,
+                                                               const PoolSel *pools, int2 *above_at)
+{
+    extern __shared__ __align__(16) float L[];
+    __shared__ int tmp[33];
+    const int c = blockIdx.x, bh = blockIdx.y;
+    const int64_t bhc = (int64_t)bh * a.Cq + c;
+    const int pid = pool[bh];
+    if (pid < 0 || sizes[bhc] <= 0) return;
+    const PoolSel &P = pools[pid];
+    if (P.coarse < 0 || !P.ok) return;
+    const int Csum = a.Ct + a.Ch + a.Cw;
+    const float *lrow = a.lut + bhc * Csum;
+    for (int e = threadIdx.x; e < Csum; e += blockDim.x) L[e] = lrow[e];
+    __syncthreads();
+    const ClusterCut cut = cuts[bhc];
+    const uint32_t key = P.prefix;
+    const int n_items = a.item_n[bh];
+    const int32_t *ids = a.item_id + (int64_t)bh * a.Pcap;
+    const int32_t *cnts = a.item_cnt + (int64_t)bh * a.Pcap;
+    int above = 0, at = 0;
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const uint32_t u = ordered_key(item_lambda(item_score(L, ids[i], a.Ch, a.Cw, a.Ct), cut, a.inv_sqrt_d));
+        above += u > key ? cnts[i] : 0;
+        at += u == key ? cnts[i] : 0;
+    }
+    int ta, tt;
+    block_excl_scan(above, tmp, ta);
+    block_excl_scan(at, tmp, tt);
+    if (threadIdx.x == 0) above_at[bhc] = make_int2(ta, tt);
+}
+
+// One CTA per pool: the keys at the cut go to the pool's rows in (head,
+// cluster) order until the mass target is met; every pooled row's Top-p count
+// becomes (keys above) + (its keys taken at the cut), then the hybrid rule.
+__global__ void __launch_bounds__(1024) eg_assign_kernel(const PoolSel *pools, const int32_t *sizes,
+                                                         const int32_t *pool, const int2 *above_at, int32_t *r_out,
+                                                         ClusterCut *cuts, int H, int group, int Cq, int N, int k_min)
+{
+    __shared__ unsigned long long utmp[33];
+    __shared__ unsigned long long carry_sh;
+    const int pid = blockIdx.x;
+    const PoolSel &P = pools[pid];
+    if (P.coarse < 0 || !P.ok) return;
+    const int ngroups = (H + group - 1) / group;
+    const int b = pid / ngroups, g = pid % ngroups;
+    const int h0 = g * group, h1 = min(H, h0 + group);
+    const unsigned long long rest = P.target - P.above_met;  // > 0: mass still needed at the cut
+    const unsigned long long per_key = (unsigned long long)llrint((double)expf(key_score(P.prefix)) * kPoolMassScale);
+    if (threadIdx.x == 0) carry_sh = 0ull;
+    __syncthreads();
+    for (int h = h0; h < h1; ++h) {
+        const int64_t bh = (int64_t)b * H + h;
+        if (pool[bh] != pid) continue;
+        for (int c0 = 0; c0 < Cq; c0 += blockDim.x) {
+            const int c = c0 + threadIdx.x;
+            const int64_t bhc = bh * Cq + c;
+            const bool in = c < Cq && sizes[bhc] > 0;
+            const int2 aa = in ? above_at[bhc] : make_int2(0, 0);
+            const unsigned long long unit = in ? (unsigned long long)sizes[bhc] * per_key : 0ull;
+            const unsigned long long v = unit * (unsigned long long)aa.y;
+            unsigned long long tot;
+            const unsigned long long ex = block_excl_scan(v, utmp, tot);
+            const unsigned long long before = carry_sh + ex;
+            if (in) {
+                int take;
+                if (before >= rest) take = 0;
+                else if (before + v <= rest || unit == 0ull) take = aa.y;
+                else take = (int)min((unsigned long long)aa.y, (rest - before + unit - 1) / unit);
+                int r = aa.x + take;
+                r = r > k_min ? r : k_min;
+                r = r < N ? r : N;
+                r_out[bhc] = r;
+                cuts[bhc].taken = -1;  // the list emission selects by count
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) carry_sh += tot;
+            __syncthreads();
+        }
     }
 }
 
@@ -455,7 +751,6 @@ __global__ void __launch_bounds__(1024) topk_kernel(const int32_t *sizes, const 
 // A key's side of the cut is its item's: each key costs one 16-bit load of its
 // item rank and one shared-memory lookup (the item's order key, or a class
 // byte when the keys are not cached).
-constexpr int kEmitPer = 8;
 
 __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int32_t *n_in, const long long *offsets,
                                                            const ClusterCut *cuts, const int32_t *coarse_hist,
@@ -463,7 +758,6 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
 {
     extern __shared__ __align__(16) float L[];
     __shared__ SelShared S;
-    __shared__ unsigned ptmp[33];
     const int c = blockIdx.x, bh = blockIdx.y;
     const int64_t bhc = (int64_t)bh * a.Cq + c;
     const int n = n_in[bhc];
@@ -530,48 +824,72 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         }
         return cls[item];
     };
+    // Key walk without block-wide scans: warp w owns a contiguous chunk of the
+    // keys (a multiple of 64).  Pass 1 counts each chunk's keys above and at
+    // the cut; after one barrier every warp knows its chunk's output base, and
+    // pass 2 walks the chunk again, 64 keys per step (two per lane), placing
+    // each key by warp ballots.
     const uint16_t *ki = a.key_item + (int64_t)bh * a.N;
-    const bool vec = (((int64_t)bh * a.N) & 7) == 0;  // 16-byte aligned rows of 8 ranks
-    int gt_run = 0, eq_run = 0;
-    for (int base = 0; base < a.N; base += kSelThreads * kEmitPer) {
-        const int j0 = base + threadIdx.x * kEmitPer;
-        unsigned gt = 0, eq = 0;
-        uint8_t k[kEmitPer];
-        if (vec && j0 + kEmitPer <= a.N) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(ki + j0);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int t = 0; t < kEmitPer; ++t) k[t] = class_of((ws[t >> 1] >> (16 * (t & 1))) & 0xffffu);
+    const bool pair = (((int64_t)bh * a.N) & 1) == 0;  // 4-byte aligned pairs of ranks
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int chunk = (((a.N + nwarps - 1) / nwarps) + 63) & ~63;
+    const int j_begin = min(a.N, warp * chunk), j_end = min(a.N, j_begin + chunk);
+    __shared__ int wgt[32], weq[32];
+    auto classes = [&](int j0, uint8_t &k0, uint8_t &k1) {
+        const int j = j0 + 2 * lane;
+        if (pair && j + 1 < j_end) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(ki + j);
+            k0 = class_of(w & 0xffffu);
+            k1 = class_of(w >> 16);
         } else {
-#pragma unroll
-            for (int t = 0; t < kEmitPer; ++t) k[t] = j0 + t < a.N ? class_of(ki[j0 + t]) : 0;
+            k0 = j < j_end ? class_of(ki[j]) : 0;
+            k1 = j + 1 < j_end ? class_of(ki[j + 1]) : 0;
         }
+    };
+    int g_cnt = 0, e_cnt = 0;
+    for (int j0 = j_begin; j0 < j_end; j0 += 64) {
+        uint8_t k0, k1;
+        classes(j0, k0, k1);
+        g_cnt += __popc(__ballot_sync(0xffffffffu, k0 == 2)) + __popc(__ballot_sync(0xffffffffu, k1 == 2));
+        e_cnt += __popc(__ballot_sync(0xffffffffu, k0 == 1)) + __popc(__ballot_sync(0xffffffffu, k1 == 1));
+    }
+    if (lane == 0) {
+        wgt[warp] = g_cnt;
+        weq[warp] = e_cnt;
+    }
+    __syncthreads();
+    unsigned g = 0, e = 0;  // keys above / at the cut before this warp's chunk
+    for (int w = 0; w < warp; ++w) {
+        g += wgt[w];
+        e += weq[w];
+    }
+    const uint32_t lt = lanemask_lt();
+    for (int j0 = j_begin; j0 < j_end; j0 += 64) {
+        uint8_t k0, k1;
+        classes(j0, k0, k1);
+        const uint32_t g0 = __ballot_sync(0xffffffffu, k0 == 2), g1 = __ballot_sync(0xffffffffu, k1 == 2);
+        const uint32_t e0 = __ballot_sync(0xffffffffu, k0 == 1), e1 = __ballot_sync(0xffffffffu, k1 == 1);
+        // keys before this lane's first key: both keys of every lower lane
+        unsigned gl = g + __popc(g0 & lt) + __popc(g1 & lt), el = e + __popc(e0 & lt) + __popc(e1 & lt);
+        const int j = j0 + 2 * lane;
 #pragma unroll
-        for (int t = 0; t < kEmitPer; ++t) {
-            gt += k[t] == 2;
-            eq += k[t] == 1;
-        }
-        unsigned tot;
-        const unsigned ex = block_excl_scan(gt | (eq << 16), ptmp, tot);
-        unsigned g = gt_run + (ex & 0xffffu), e = eq_run + (ex >> 16);
-#pragma unroll
-        for (int t = 0; t < kEmitPer; ++t) {
-            const int j = j0 + t;
-            if (k[t] == 2) {
-                const unsigned slot = g + (e < (unsigned)need ? e : (unsigned)need);
-                if (slot < (unsigned)n) out[slot] = j;
+        for (int t = 0; t < 2; ++t) {
+            const uint8_t kt = t ? k1 : k0;
+            if (kt == 2) {
+                const unsigned slot = gl + (el < (unsigned)need ? el : (unsigned)need);
+                if (slot < (unsigned)n) out[slot] = j + t;
                 else set_error(a.err, kErrRange, 0x300 + c);
-                ++g;
-            } else if (k[t] == 1) {
-                if (e < (unsigned)need) {
-                    if (g + e < (unsigned)n) out[g + e] = j;
+                ++gl;
+            } else if (kt == 1) {
+                if (el < (unsigned)need) {
+                    if (gl + el < (unsigned)n) out[gl + el] = j + t;
                     else set_error(a.err, kErrRange, 0x300 + c);
                 }
-                ++e;
+                ++el;
             }
         }
-        gt_run += tot & 0xffffu;
-        eq_run += tot >> 16;
+        g += __popc(g0) + __popc(g1);
+        e += __popc(e0) + __popc(e1);
     }
 }
 
@@ -582,11 +900,17 @@ static size_t sel_smem(int Csum) { return (size_t)((Csum + 3) & ~3) * sizeof(flo
 cudaError_t select_configure()
 {
     static_assert(kItemCache * 4 >= kMaxItems, "the 64 KB region must hold a class byte per item");
+    const int max_csum = kMaxBlocks + 2 > 3 * kMaxClusters ? kMaxBlocks + 2 : 3 * kMaxClusters;
     cudaError_t e = cudaFuncSetAttribute(emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sel_smem(3 * kMaxClusters));
+                                         (int)sel_smem(max_csum));
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(topp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)sel_smem(3 * kMaxClusters));
+    e = cudaFuncSetAttribute(eg_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(3 * kMaxClusters * sizeof(float)));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(eg_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(3 * kMaxClusters * sizeof(float)));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(topp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem(max_csum));
 }
 
 // -------------------------------------------------------------- launchers
@@ -631,14 +955,21 @@ void launch_emit(const SelArgs &a, const int32_t *n_in, const long long *offsets
     count_launches(1);
 }
 
-// Bytes of per-cluster selection state (cut record + coarse histogram).
+// Bytes of per-cluster selection state (cut record + coarse histogram) and,
+// with EG-Sparse routing, of the head entropies, pool ids, per-cluster cut
+// counts and per-pool histograms.
 size_t selection_state_bytes(int64_t clusters) { return (size_t)clusters * (sizeof(ClusterCut) + kBuckets * 4); }
+size_t eg_state_bytes(int64_t B, int64_t H, int64_t Cq, int group)
+{
+    const int64_t pools = B * ((H + group - 1) / group);
+    return (size_t)(B * H * 8 + B * H * Cq * 8 + 256) + (size_t)pools * sizeof(PoolSel);
+}
 
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
                    const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch,
                    int Cw, int BH, float top_p, float inv_sqrt_d, int k_min, int32_t *err, const int32_t *sizes,
                    int32_t *r, int32_t *n, int32_t *kh, long long *offsets, int32_t *indices, int online,
-                   void *state, cudaStream_t st)
+                   void *state, int B, float eg_tau, int eg_group, void *eg_state, int whole_items, cudaStream_t st)
 {
     SelArgs a;
     a.lut = lut;
@@ -657,10 +988,35 @@ void run_selection(const float *lut, const int32_t *codes, const int32_t *item_i
     a.top_p = top_p;
     a.inv_sqrt_d = inv_sqrt_d;
     a.k_min = k_min;
+    a.whole_items = whole_items;
     a.err = err;
     ClusterCut *cuts = reinterpret_cast<ClusterCut *>(state);
     int32_t *coarse_hist = reinterpret_cast<int32_t *>(cuts + (int64_t)BH * Cq);
     launch_topp(a, r, cuts, coarse_hist, st);
+    if (eg_tau > 0.f && top_p < 1.0f) {
+        // EG-Sparse: entropies, routing, then the pooled Top-p of every group
+        const int H = BH / B;
+        const int npools = B * ((H + eg_group - 1) / eg_group);
+        float *entropy = reinterpret_cast<float *>(eg_state);
+        int32_t *pool = reinterpret_cast<int32_t *>(entropy + BH);
+        int2 *above_at = reinterpret_cast<int2 *>(pool + BH);
+        PoolSel *pools = reinterpret_cast<PoolSel *>(
+            (reinterpret_cast<uintptr_t>(above_at + (int64_t)BH * Cq) + 255) & ~(uintptr_t)255);
+        cudaMemsetAsync(pools, 0, (size_t)npools * sizeof(PoolSel), st);
+        eg_route_kernel<<<B, 1024, 0, st>>>(cuts, sizes, entropy, pool, H, Cq, N, eg_tau, eg_group);
+        const size_t lsm = (size_t)((Ct + Ch + Cw + 3) & ~3) * sizeof(float);
+        const dim3 grid(Cq, BH);
+        eg_hist_kernel<<<grid, kSelThreads, lsm, st>>>(a, cuts, sizes, pool, pools, -1, 11);
+        eg_pick_kernel<<<npools, kSelThreads, 0, st>>>(pools, top_p, -1, 11, err);
+        const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
+        for (int i = 0; i < 3; ++i) {
+            eg_hist_kernel<<<grid, kSelThreads, lsm, st>>>(a, cuts, sizes, pool, pools, shifts[i], widths[i]);
+            eg_pick_kernel<<<npools, kSelThreads, 0, st>>>(pools, top_p, shifts[i], widths[i], err);
+        }
+        eg_count_kernel<<<grid, kSelThreads, lsm, st>>>(a, cuts, sizes, pool, pools, above_at);
+        eg_assign_kernel<<<npools, 1024, 0, st>>>(pools, sizes, pool, above_at, r, cuts, H, eg_group, Cq, N, k_min);
+        count_launches(11);
+    }
     launch_topk(sizes, r, n, kh, offsets, BH, Cq, N, online, st);
     launch_emit(a, n, offsets, cuts, coarse_hist, indices, st);
 }

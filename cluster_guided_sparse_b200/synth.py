@@ -63,6 +63,12 @@ class Workload:
     label_block: Optional[tuple] = None
     # ClusterAttention variant: compensate excluded key clusters through their mean
     compensate: int = 0
+    # EG-Sparse routing: entropy threshold (0 = off) and head group size
+    eg_tau: float = 0.0
+    eg_group: int = 1
+    # VMoBA block-granular selection: 0 off, 1/2/3 = 1D/2D/3D key blocks of block_dims
+    block_kind: int = 0
+    block_dims: tuple = (4, 4, 4)
 
     @property
     def torch_dtype(self):

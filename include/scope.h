@@ -108,7 +108,38 @@ typedef struct {
  *                  m_ck members of key cluster k missing from query cluster
  *                  c's list add m_ck * e^{q.mu_k/sqrt(D)} to the softmax
  *                  denominator and that times the mean value to the
- *                  numerator. */
+ *                  numerator.
+ *   eg_tau, eg_group  EG-Sparse routing ("EG-Sparse", abstract: low-entropy
+ *                  heads go to a grouped cross-head pool, high-entropy heads
+ *                  keep per-row selection).  eg_tau <= 0: off (plain SCOPE
+ *                  selection).  Otherwise a head's entropy E_h is the
+ *                  query-weighted mean entropy of its clusters' proxy
+ *                  softmax rows over ln N (0..1); heads with E_h < eg_tau
+ *                  are grouped eg_group at a time in index order (per batch
+ *                  entry, 1 <= eg_group <= 64), and a group's low-entropy
+ *                  heads take their Top-p counts from one pool: every (head,
+ *                  cluster, key) entry competes by its row's proxy
+ *                  probability and the shortest prefix reaching top_p of
+ *                  the pool's mass (each entry weighing its cluster's query
+ *                  count) is kept.  k_min, the online Top-k and the lists
+ *                  then follow as for the other heads.
+ *   block_kind     VMoBA block-granular selection ("VMoBA: Mixture-of-Block
+ *                  Attention for Video Diffusion Models", abstract: a
+ *                  layer-wise recurrent 1D-2D-3D block partition, and blocks
+ *                  chosen by a threshold on their cumulative similarity).
+ *                  0: off (per-key SCOPE selection).  1, 2, 3: keys are
+ *                  grouped into blocks -- 1: runs of block_t*block_h*block_w
+ *                  tokens in raster order; 2: block_h x block_w tiles inside
+ *                  each frame; 3: block_t x block_h x block_w cubes (ragged
+ *                  edges; the caller cycles the kind with the layer index) --
+ *                  in place of the key-subspace clustering.  Each block is
+ *                  scored for query cluster c by q_c . (mean of its rotated
+ *                  keys); blocks are kept by descending score until their
+ *                  size-weighted softmax(score/sqrt(D)) mass reaches top_p,
+ *                  whole blocks only (blocks tied with the last kept one are
+ *                  kept too).  Needs a grid, at most 16384 blocks, k_min = 0,
+ *                  online_topk = 0, eg_tau = 0 and no fixed_cluster_size;
+ *                  c_t, c_h, c_w are not used. */
 typedef struct {
     int32_t d_t, d_h, d_w;
     double theta;
@@ -120,6 +151,10 @@ typedef struct {
     int32_t online_topk;
     int32_t fixed_cluster_size;
     int32_t compensate;
+    float eg_tau;
+    int32_t eg_group;
+    int32_t block_kind;
+    int32_t block_t, block_h, block_w;
 } scope_params;
 
 typedef struct scope_plan_s scope_plan_t; /* opaque host handle */
@@ -188,7 +223,9 @@ typedef enum {
     SCOPE_VIEW_OFFSETS = 15,    /* i64  [B*H*c_q+1] list starts in INDICES */
     SCOPE_VIEW_INDICES = 16,    /* i32  [capacity] selected keys, ascending per cluster */
     SCOPE_VIEW_ERROR = 17,      /* i32  [4] device error word              */
-    SCOPE_VIEW_COUNT = 18
+    SCOPE_VIEW_EG_ENTROPY = 18, /* f32  [B,H] EG-Sparse head entropy (eg_tau > 0) */
+    SCOPE_VIEW_EG_POOL = 19,    /* i32  [B,H] pool (group) of a routed head, -1 if not routed */
+    SCOPE_VIEW_COUNT = 20
 } scope_view_id;
 
 typedef struct {

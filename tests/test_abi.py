@@ -68,6 +68,11 @@ def test_workspace_bytes_counts_list_capacity(L):
     (dict(fixed_cluster_size=64), 1, "grid"),
     (dict(compensate=2), 1, "compensate"),
     (dict(compensate=1), 1, "compensate"),
+    (dict(eg_tau=0.5, eg_group=0), 1, "eg_group"),
+    (dict(eg_tau=-0.1), 1, "eg_tau"),
+    (dict(block_kind=5), 1, "block_kind"),
+    (dict(block_kind=3, block_t=2, block_h=4, block_w=8), 1, "k_min"),
+    (dict(block_kind=3, block_t=0, block_h=4, block_w=8, k_min=0, online_topk=0), 1, "block_t"),
 ])
 def test_bad_params_rejected_on_host(L, mut, code, msg):
     p, g = P(**mut)
@@ -177,3 +182,12 @@ def test_selftest_wait_timeout_checks_arguments(L):
     assert L.scope_selftest_wait_timeout(ctypes.c_void_p(FAKE), 10, None) == 1
     assert "wait_cycles" in L.scope_last_error().decode()
     assert L.scope_selftest_wait_timeout(ctypes.c_void_p(FAKE), 5_000_000_000, None) == 1
+
+
+def test_block_mode_block_count_limit(L):
+    p, g = P(block_kind=1, block_t=1, block_h=1, block_w=1, k_min=0, online_topk=0, grid=(64, 64, 64))
+    q = T(N=64 * 64 * 64, H=1)
+    st, err = plan_status(L, q, q, p, g)
+    assert st == 1 and "blocks >" in err  # 262 144 one-token blocks > 16 384
+    p, g = P(block_kind=3, block_t=4, block_h=4, block_w=4, k_min=0, online_topk=0, grid=(64, 64, 64))
+    assert L.scope_plan_workspace_bytes(ctypes.byref(q), ctypes.byref(g), ctypes.byref(p)) > 0  # 4096 blocks
