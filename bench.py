@@ -402,6 +402,10 @@ def workload_of(args):
         w = w.with_(top_p=args.top_p)
     if getattr(args, "compensate", False):
         w = w.with_(compensate=1)
+    if getattr(args, "block_kind", None):
+        w = w.with_(block_kind=args.block_kind, k_min=0, online_topk=0)
+    if getattr(args, "eg_tau", None):
+        w = w.with_(eg_tau=args.eg_tau, eg_group=args.eg_group)
     return w
 
 
@@ -486,6 +490,9 @@ def run_scope(args, world, rank, local):
     gather_ms = max_over_ranks(statistics.mean(e[2].elapsed_time(e[3]) for e in ev), world)
     call_median_ms = max_over_ranks(statistics.median(e[0].elapsed_time(e[3]) for e in ev), world)
 
+    # rows the final tensor-core query assignment sent to the fp64 re-check
+    fix_rows = int(pl.view("fixup")[0]) if w.c_q >= 128 and w.fixed_cluster_size == 0 and w.block_kind == 0 else 0
+    fix_rows = int(sum_over_ranks(fix_rows, world))
     # algorithmic attention flops of one launch: 4 d sum_c |c| n_c (this rank's heads)
     sizes = pl.view("q_sizes").to(torch.int64)
     n = pl.view("n").to(torch.int64)
@@ -531,29 +538,46 @@ def run_scope(args, world, rank, local):
     dens_h = [by_head[h][2] for h in range(w.H)]
     del od
 
-    # end to end through the public API with host buffers: Q and K go first
-    # (scope_plan reads them); V is only read by scope_attn, so its copy runs
-    # on a side stream while the plan computes.
+    # end to end through the public API with host buffers.  Heads are
+    # independent (SCOPE clusters and selects per head), so the call runs on
+    # chunks of heads: while the device plans and attends over chunk i, the
+    # copy stream brings chunk i + 1's Q, K, V in and chunk i - 1's O out.
+    # Every chunk is a scope_plan + scope_attn on head slices of the same
+    # tensors (views, no repacking); the timed region spans the first H2D
+    # copy to the last D2H copy.
     e2e = []
     oh = torch.empty(qd.shape, dtype=torch.bfloat16).pin_memory()
-    side = torch.cuda.Stream(dev)
+    h_loc = qd.shape[1]
+    n_chunks = max(1, min(args.e2e_chunks, h_loc))
+    bounds = [(h_loc * i) // n_chunks for i in range(n_chunks + 1)]
+    chunks = [(bounds[i], bounds[i + 1]) for i in range(n_chunks) if bounds[i + 1] > bounds[i]]
+    copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ws_e2e = torch.empty(max(scope.workspace_bytes(qd[:, h0:h1], params, grid) for h0, h1 in chunks),
+                         dtype=torch.uint8, device=dev) if len(chunks) > 1 else ws
     for i in range(args.warmup + args.steps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        qk_in, v_in = torch.cuda.Event(), torch.cuda.Event()
         barrier(world)
         torch.cuda.synchronize()
         a.record(stream)
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        qk_in.record(stream)
-        side.wait_event(qk_in)
-        with torch.cuda.stream(side):
-            vd.copy_(vh, non_blocking=True)
-            v_in.record(side)
-        pl = scope.plan(qd, kd, params, grid, workspace=ws)
-        stream.wait_event(v_in)
-        scope.attn(qd, kd, vd, pl, out=o)
-        oh.copy_(o, non_blocking=True)
+        copy_in.wait_stream(stream)
+        landed, done = [], []
+        for (h0, h1) in chunks:
+            with torch.cuda.stream(copy_in):
+                for dev_t, host_t in ((qd, qh), (kd, kh), (vd, vh)):
+                    dev_t[:, h0:h1].copy_(host_t[:, h0:h1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy_in)
+                landed.append(ev)
+        for c, (h0, h1) in enumerate(chunks):
+            stream.wait_event(landed[c])
+            pl = scope.plan(qd[:, h0:h1], kd[:, h0:h1], params, grid, workspace=ws_e2e)
+            scope.attn(qd[:, h0:h1], kd[:, h0:h1], vd[:, h0:h1], pl, out=o[:, h0:h1])
+            ev = torch.cuda.Event()
+            ev.record(stream)
+            copy_out.wait_event(ev)
+            with torch.cuda.stream(copy_out):
+                oh[:, h0:h1].copy_(o[:, h0:h1], non_blocking=True)
+        stream.wait_stream(copy_out)
         b.record(stream)
         torch.cuda.synchronize()
         if i >= args.warmup:
@@ -581,6 +605,10 @@ def run_scope(args, world, rank, local):
         "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.N, "heads": w.H, "head_dim": w.D,
                    "top_p": w.top_p, "online_topk": bool(w.online_topk), "compensate": bool(w.compensate),
+                   "selection": ("VMoBA %dD blocks %s" % (w.block_kind, "x".join(map(str, w.block_dims)))
+                                 if w.block_kind else
+                                 "EG-Sparse tau %g, groups of %d" % (w.eg_tau, w.eg_group) if w.eg_tau > 0 else
+                                 "per-key (SCOPE)"),
                    "l2": f"inputs {3 * w.B * w.H * w.N * w.D * 2 / 1e9:.2g} GB vs 126 MB L2, no flush",
                    "parallelism": "single GPU" if world == 1 else
                    f"heads round-robin over {world} GPUs" + (", O all-gathered" if gather else "")},
@@ -591,6 +619,7 @@ def run_scope(args, world, rank, local):
                                   "psnr_db_mean": statistics.mean(psnr_fin) if psnr_fin else None,
                                   "psnr_db_min": min(psnr_h), "rel_l2_per_head": [round(x, 5) for x in rel_h],
                                   "psnr_db_per_head": [round(x, 2) for x in psnr_h]},
+        "query_fixup_rows": fix_rows, "query_fixup_fraction": fix_rows / float(w.B * w.H * w.N),
         "tile_tflops": tile_tf, "tile_frac_of_sustained": tile_tf / bf16_sus,
         "own_dense_ms": dense_ms, "speedup_vs_own_dense": dense_ms / ms_per_call,
         "roofline": {"kernel": "sparse attention (scope_attn, attn_tc_kernel)", "bound": "tensor",
@@ -599,7 +628,8 @@ def run_scope(args, world, rank, local):
                      "algorithmic_bytes": attn_bytes_local,
                      "traffic_over_algorithmic": None if traffic is None else traffic / attn_bytes_local,
                      "peak_source": f"{src} bf16 sustained", "algorithmic_tflop_per_call": attn_flops / 1e12},
-        "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "e2e": {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "head_chunks": len(chunks)},
         "gpu_launches": launches,
         "clocks": clk,
         "cpu_baseline": cpu,
@@ -616,8 +646,13 @@ def main():
     ap.add_argument("--workload", default="hunyuan720p", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--top-p", type=float, default=None, help="override the workload's Top-p")
     ap.add_argument("--compensate", action="store_true", help="ClusterAttention compensation (unstructured only)")
+    ap.add_argument("--block-kind", type=int, default=None, help="VMoBA block selection: 1/2/3 = 1D/2D/3D blocks")
+    ap.add_argument("--eg-tau", type=float, default=None, help="EG-Sparse entropy threshold (0 = off)")
+    ap.add_argument("--eg-group", type=int, default=4)
     ap.add_argument("--no-gather", action="store_true", help="N > 1: leave the output heads sharded")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=4,
+                    help="head chunks of the end-to-end call (copies of one chunk overlap compute of another)")
     args = ap.parse_args()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         sys.exit(relaunch(args.gpus))

@@ -45,6 +45,15 @@ struct RowStrides {
     __host__ __device__ __forceinline__ int64_t row(int64_t bh, int64_t n) const { return bh_off(bh) + n * sN; }
 };
 
+// Rows of up to four problems that a tensor-core assignment left to the
+// fp64 re-decision: per problem a device counter and list of bh * N + n.
+struct FixBatch {
+    KmProblem p[4];
+    const int32_t *list[4];
+    const int32_t *count[4];
+    int n;
+};
+
 struct KmBatch {
     KmProblem p[4];
     int count;

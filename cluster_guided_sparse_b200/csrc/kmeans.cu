@@ -184,13 +184,14 @@ static size_t direct_smem(int dn)
 // warps' winners then meet in shared memory.
 constexpr int kFixWarps = 8;
 
-__global__ void __launch_bounds__(kFixWarps * 32) km_fixup_kernel(KmProblem P, int N, int D, const int32_t *fix_list,
-                                                                  const int32_t *fix_count)
+__global__ void __launch_bounds__(kFixWarps * 32) km_fixup_kernel(FixBatch fb, int N, int D)
 {
     __shared__ double wbest[kFixWarps];
     __shared__ int warg[kFixWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int count = *fix_count;
+    const KmProblem &P = fb.p[blockIdx.y];  // one problem (and its list) per grid row
+    const int32_t *fix_list = fb.list[blockIdx.y];
+    const int count = *fb.count[blockIdx.y];
     const int C = P.C, dn = P.dim_n;
     for (int w = blockIdx.x; w < count; w += gridDim.x) {
         const int gid = fix_list[w];
@@ -576,11 +577,11 @@ void launch_km_assign_direct(const KmBatch &b, int BH, int N, int D, cudaStream_
     count_launches(1);
 }
 
-void km_fixup_launch(const KmProblem &P, int BH, int N, int D, const int32_t *fix_list, const int32_t *fix_count,
-                     cudaStream_t st)
+// One launch re-decides the listed rows of every problem of the batch.
+void km_fixup_launch(const FixBatch &fb, int N, int D, cudaStream_t st)
 {
-    (void)BH;
-    km_fixup_kernel<<<148 * 8, kFixWarps * 32, 0, st>>>(P, N, D, fix_list, fix_count);
+    if (fb.n == 0) return;
+    km_fixup_kernel<<<dim3(148 * 8 / fb.n, fb.n), kFixWarps * 32, 0, st>>>(fb, N, D);
     count_launches(1);
 }
 

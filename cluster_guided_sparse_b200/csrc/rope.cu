@@ -65,8 +65,8 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, flo
 template <typename TIn>
 __global__ void __launch_bounds__(256) rope_apply_kernel(
     const TIn *__restrict__ in, RowStrides rs, __nv_bfloat16 *__restrict__ out, float *__restrict__ norm2,
-    uint32_t *__restrict__ maxabs, const double2 *__restrict__ tab, int64_t rows, int N, int D,
-    int Hh, int W, int dt, int dh, int maxL, int maxP, int use_rope)
+    float4 *__restrict__ sub2, uint32_t *__restrict__ maxabs, const double2 *__restrict__ tab, int64_t rows, int N,
+    int D, int Hh, int W, int dt, int dh, int maxL, int maxP, int use_rope)
 {
     __shared__ float bmax[8];
     const int tpr = D >> 3;  // 8 or 16 threads per row (D is 64 or 128)
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(
     const int64_t row = gid >> sh;  // < rows < 2^31
     const int c8 = (int)(gid & (tpr - 1));
     const bool valid = row < rows;
-    float ss = 0.f, mx = 0.f;
+    float ss = 0.f, mx = 0.f, nt = 0.f, nh = 0.f, nw = 0.f;  // row sum of squares and its t, h, w parts
     if (valid) {
         float x[8];
         load8<TIn>(in + rs.row(row / N, row % N) + c8 * 8, x);
@@ -108,15 +108,27 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(
             o[p].x = __double2bfloat16(y[2 * p]);
             o[p].y = __double2bfloat16(y[2 * p + 1]);
             const float2 r = __bfloat1622float2(o[p]);
-            ss = fmaf(r.x, r.x, ss);
-            ss = fmaf(r.y, r.y, ss);
+            const float q2 = fmaf(r.y, r.y, r.x * r.x);  // the pair shares its block (blocks have even widths)
+            ss += q2;
+            const int d = c8 * 8 + 2 * p;
+            nt += d < dt ? q2 : 0.f;
+            nh += (d >= dt && d < dt + dh) ? q2 : 0.f;
+            nw += d >= dt + dh ? q2 : 0.f;
             mx = fmaxf(mx, fmaxf(fabsf(r.x), fabsf(r.y)));
         }
         *reinterpret_cast<uint4 *>(out + row * D + c8 * 8) = *reinterpret_cast<const uint4 *>(o);
     }
     // Row norm over the tpr lanes that share the row (tpr divides 32).
-    for (int o = tpr >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    for (int o = tpr >> 1; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        nt += __shfl_xor_sync(0xffffffffu, nt, o);
+        nh += __shfl_xor_sync(0xffffffffu, nh, o);
+        nw += __shfl_xor_sync(0xffffffffu, nw, o);
+    }
     if (norm2 && valid && c8 == 0) norm2[row] = ss;
+    // squared norms of the (t, h, w) blocks of the stored row, for the key
+    // subspaces' assignment error bound
+    if (sub2 && valid && c8 == 0) sub2[row] = make_float4(nt, nh, nw, ss);
     // max |x| per (batch, head): the block's rows nearly always belong to one
     // head, whose maximum then takes one atomic (per-warp atomics on one word
     // would serialise); a block that straddles two heads updates per thread.
@@ -144,7 +156,7 @@ void launch_rope_table(double2 *tab, int T, int Hh, int W, int dt, int dh, int d
 }
 
 void launch_rope_apply(const void *in, const RowStrides &rs, bool in_f32, __nv_bfloat16 *out, float *norm2,
-                       uint32_t *maxabs,
+                       float4 *sub2, uint32_t *maxabs,
                        const double2 *tab, int64_t rows, int N, int D, int Hh, int W, int dt, int dh,
                        int maxL, int maxP, int use_rope, cudaStream_t st)
 {
@@ -152,10 +164,10 @@ void launch_rope_apply(const void *in, const RowStrides &rs, bool in_f32, __nv_b
     const int64_t blocks = (threads + 255) / 256;
     if (in_f32)
         rope_apply_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
-            (const float *)in, rs, out, norm2, maxabs, tab, rows, N, D, Hh, W, dt, dh, maxL, maxP, use_rope);
+            (const float *)in, rs, out, norm2, sub2, maxabs, tab, rows, N, D, Hh, W, dt, dh, maxL, maxP, use_rope);
     else
         rope_apply_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)in, rs, out, norm2, maxabs, tab, rows, N, D, Hh, W, dt, dh, maxL, maxP,
+            (const __nv_bfloat16 *)in, rs, out, norm2, sub2, maxabs, tab, rows, N, D, Hh, W, dt, dh, maxL, maxP,
             use_rope);
     count_launches(1);
 }

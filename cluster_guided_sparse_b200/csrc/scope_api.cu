@@ -15,8 +15,11 @@
 namespace scope {
 // kernels.cu launchers
 void launch_rope_table(double2 *, int, int, int, int, int, int, double, int, int, cudaStream_t);
-void launch_rope_apply(const void *, const RowStrides &, bool, __nv_bfloat16 *, float *, uint32_t *, const double2 *,
-                       int64_t, int, int, int, int, int, int, int, int, int, cudaStream_t);
+void launch_rope_apply(const void *, const RowStrides &, bool, __nv_bfloat16 *, float *, float4 *, uint32_t *,
+                       const double2 *, int64_t, int, int, int, int, int, int, int, int, int, cudaStream_t);
+void km_fixup_launch(const FixBatch &, int, int, cudaStream_t);
+bool launch_km_assign_keys_tc(const KmProblem *, __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, const float4 *,
+                              int32_t *, int32_t *, cudaStream_t);
 void launch_to_bf16(const float *, const RowStrides &, __nv_bfloat16 *, int64_t, int, int, cudaStream_t);
 cudaError_t km_configure();
 void launch_km_init(const KmBatch &, int, int, int, uint32_t, cudaStream_t);
@@ -93,7 +96,7 @@ struct Layout {
     int Cq, C[3], ds[3], off[3], Csum, P, Pcap, nblk, max_work, maxL, maxP;
     bool f32, bisect;
     int64_t cap;
-    size_t qr, kr, qnorm, tab, stats, maxabs, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist, q_tsum;
+    size_t qr, kr, qnorm, ksub2, kchi, kclo, kfix, tab, stats, maxabs, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist, q_tsum;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3], k_tsum[3];
     size_t sel_state, eg_state, lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
     size_t bis_order, bis_delta, bis_aux, q_chi, q_clo, q_sums, k_sums[3], sums_bytes, lse, vmean;
@@ -332,6 +335,10 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.qr = take(cur, BH * N * D * 2);
     L.kr = take(cur, BH * N * D * 2);
     L.qnorm = take(cur, BH * N * 4);
+    L.ksub2 = take(cur, BH * N * 16);
+    L.kchi = take(cur, BH * 128 * D * 2);
+    L.kclo = take(cur, BH * 128 * D * 2);
+    L.kfix = take(cur, 3 * (4 + BH * N) * 4);
     L.tab = take(cur, (size_t)3 * L.maxL * L.maxP * 16);
     L.stats = take(cur, 64);
     L.maxabs = take(cur, 2 * BH * 4);
@@ -454,10 +461,11 @@ static void rope_both(const Layout &L, char *ws, const scope_tensor *q, const sc
         launch_rope_table(at<double2>(ws, L.tab), g->T, g->Hh, g->W, p->d_t, p->d_h, p->d_w, p->theta, L.maxL, L.maxP,
                           st);
     const int Hh = rope ? g->Hh : 1, W = rope ? g->W : 1;
-    launch_rope_apply(q->ptr, rows_of(q), L.f32, at<__nv_bfloat16>(ws, L.qr), at<float>(ws, L.qnorm), maxabs,
+    launch_rope_apply(q->ptr, rows_of(q), L.f32, at<__nv_bfloat16>(ws, L.qr), at<float>(ws, L.qnorm), nullptr, maxabs,
                       at<double2>(ws, L.tab), L.BH * L.N, (int)L.N, (int)L.D, Hh, W, p->d_t, p->d_h, L.maxL, L.maxP,
                       rope ? 1 : 0, st);
-    launch_rope_apply(k->ptr, rows_of(k), L.f32, at<__nv_bfloat16>(ws, L.kr), nullptr, maxabs + L.BH, at<double2>(ws, L.tab),
+    launch_rope_apply(k->ptr, rows_of(k), L.f32, at<__nv_bfloat16>(ws, L.kr), nullptr,
+                      L.ksub2 ? at<float4>(ws, L.ksub2) : nullptr, maxabs + L.BH, at<double2>(ws, L.tab),
                       L.BH * L.N, (int)L.N, (int)L.D, Hh, W, p->d_t, p->d_h, L.maxL, L.maxP, rope ? 1 : 0, st);
 }
 
@@ -565,15 +573,41 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
     int32_t *fix_count = at<int32_t>(ws, L.fix);
     int32_t *fix_list = fix_count + 4;
     bool tc_ok = true;
+    // key subspaces on the tensor cores when their centroids fit one
+    // 128-column block-diagonal chunk
+    const bool tc_k = keys.count == 3 && L.C[0] + L.C[1] + L.C[2] <= 128;
     auto assign = [&]() {
+        if (tc_k)
+            tc_ok = tc_ok && launch_km_assign_keys_tc(keys.p, at<__nv_bfloat16>(ws, L.kchi),
+                                                      at<__nv_bfloat16>(ws, L.kclo), BH, N, D,
+                                                      at<float4>(ws, L.ksub2), at<int32_t>(ws, L.kfix),
+                                                      at<int32_t>(ws, L.stats) + 4, s);
         if (tc_q) {
-            if (keys.count) launch_km_assign_direct(keys, BH, N, D, s);
-            tc_ok = tc_ok && launch_km_assign_tc(all.p[3], at<__nv_bfloat16>(ws, L.q_chi),
+            if (keys.count && !tc_k) launch_km_assign_direct(keys, BH, N, D, s);
+            tc_ok = tc_ok && launch_km_assign_tc(qonly.p[0], at<__nv_bfloat16>(ws, L.q_chi),
                                                  at<__nv_bfloat16>(ws, L.q_clo), BH, N, D, at<float>(ws, L.qnorm),
                                                  fix_list, fix_count, at<int32_t>(ws, L.stats) + 4, s);
         } else {
-            launch_km_assign_direct(all, BH, N, D, s);
+            launch_km_assign_direct(keys.count && !tc_k ? all : qonly, BH, N, D, s);
         }
+        // fp64 re-decision of every tensor-core-assigned row inside its margin, one launch
+        FixBatch fb{};
+        if (tc_q) {
+            fb.p[fb.n] = qonly.p[0];
+            fb.list[fb.n] = fix_list;
+            fb.count[fb.n] = fix_count;
+            ++fb.n;
+        }
+        if (tc_k)
+            for (int k = 0; k < 3; ++k)
+                if (keys.p[k].C > 1) {
+                    int32_t *kc = at<int32_t>(ws, L.kfix) + (int64_t)k * (4 + (int64_t)BH * N);
+                    fb.p[fb.n] = keys.p[k];
+                    fb.count[fb.n] = kc;
+                    fb.list[fb.n] = kc + 4;
+                    ++fb.n;
+                }
+        km_fixup_launch(fb, N, D, s);
     };
     cudaMemsetAsync(ws + L.q_sums, 0, L.sums_bytes, s);
     launch_km_init(all, BH, N, D, p->init_seed, s);
@@ -788,6 +822,7 @@ extern "C" scope_status scope_plan_view(const scope_plan_t *plan, int which, sco
     case SCOPE_VIEW_OFFSETS: set(L.offsets, SCOPE_I64, 1, L.BH * L.Cq + 1, 0, 0, 0); break;
     case SCOPE_VIEW_INDICES: set(L.indices, SCOPE_I32, 1, L.cap, 0, 0, 0); break;
     case SCOPE_VIEW_ERROR: set(L.stats + 16, SCOPE_I32, 1, 4, 0, 0, 0); break;
+    case SCOPE_VIEW_FIXUP: set(L.fix, SCOPE_I32, 1, 1, 0, 0, 0); break;
     case SCOPE_VIEW_EG_ENTROPY:
         if (!L.eg) return fail(SCOPE_EINVAL, "no EG-Sparse routing in this plan (eg_tau = 0)");
         set(L.eg_state, SCOPE_F32, 2, B, H, 0, 0);

@@ -225,7 +225,8 @@ typedef enum {
     SCOPE_VIEW_ERROR = 17,      /* i32  [4] device error word              */
     SCOPE_VIEW_EG_ENTROPY = 18, /* f32  [B,H] EG-Sparse head entropy (eg_tau > 0) */
     SCOPE_VIEW_EG_POOL = 19,    /* i32  [B,H] pool (group) of a routed head, -1 if not routed */
-    SCOPE_VIEW_COUNT = 20
+    SCOPE_VIEW_FIXUP = 20,      /* i32  [1] rows the last tensor-core query assignment sent to the fp64 re-check */
+    SCOPE_VIEW_COUNT = 21
 } scope_view_id;
 
 typedef struct {
@@ -272,12 +273,13 @@ int scope_version(void);
 /* [dim_off, dim_off + dim_n) of x with scope_plan's strided init, tie      */
 /* rule, empty-cluster rule, final assign and per-head fixed-point centroid */
 /* sums, assigning by the fp32 direct-form distance.  Given the plan's      */
-/* rotated rows and C < 128 (the plan's key subspaces, and its queries at   */
-/* fewer than 128 clusters) its labels and centroids equal the plan's.  At  */
-/* C >= 128 the plan decides query labels exactly (tensor cores plus an     */
-/* fp64 re-decision of near-ties), while this entry point keeps the fp32    */
-/* direct form: a label can then differ where a row's two nearest centroids */
-/* lie within fp32 rounding of each other, and later rounds follow from it. */
+/* rotated queries and C < 128 its labels and centroids equal the plan's    */
+/* query clustering.  Where the plan assigns on the tensor cores (queries   */
+/* at C >= 128; key subspaces whose clusters fit one 128-column chunk) it   */
+/* decides labels exactly (certified margin, fp64 re-decision of near-ties) */
+/* while this entry point keeps the fp32 direct form: a label can then      */
+/* differ where a row's two nearest centroids lie within fp32 rounding of   */
+/* each other, and later rounds follow from it.                             */
 /*   x          bf16 [B,H,N,D] device, D in {64, 128} (e.g. post-RoPE rows). */
 /*   labels     int32 [B,H,N] device, written (final assign).               */
 /*   centroids  f32 [B,H,C,dim_n] device, written (after the last update).  */

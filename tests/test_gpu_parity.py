@@ -300,7 +300,8 @@ def test_bisection_small_shapes(N, D, H):
 # ClusterAttention compensation: every excluded key enters through its key
 # cluster's mean key and value (the oracle's attention_rows_comp, reading R16),
 # fed the device's own rotated rows, key-cluster labels and lists.
-@pytest.mark.parametrize("N,D,H,p", [(4096, 64, 2, 0.9), (4096, 64, 1, 0.5), (512, 128, 1, 0.9)])
+@pytest.mark.parametrize("N,D,H,p", [(4096, 64, 2, 0.9), (4096, 64, 1, 0.5), (512, 128, 1, 0.9),
+                                     (65536, 64, 1, 0.9)])  # the benchmarked shape: 1024 key leaves
 def test_compensation_parity(N, D, H, p):
     w = synth.WORKLOADS["unstructured"].with_(N=N, D=D, H=H, d_split=(D, 0, 0), components=16, k_min=32,
                                                config_id=170 + N + D, c_q=N // 64, c_sub=(N // 64, 1, 1),

@@ -34,11 +34,22 @@ def test_noalloc_kmeans_matches_plan_twice():
         kcent = torch.full_like(ref_h_cent, float("nan"))
         scope.kmeans_noalloc(kr, d_t, d_h, w.c_sub[1], w.iters, 0, klab, kcent)
         torch.cuda.synchronize()
-        # same kernels, same per-head fixed-point scale: identical results
+        # queries: the same kernels and per-head fixed-point scale as the plan's
+        # (32 clusters, direct form): identical results
         assert torch.equal(lab, ref_q_lab)
-        assert torch.equal(klab, ref_h_lab)
         assert torch.equal(cent, ref_q_cent)
-        assert torch.equal(kcent, ref_h_cent)
+        # key subspace h: the plan decides labels exactly on the tensor cores,
+        # this entry point by the fp32 direct form; they may differ only on rows
+        # whose two nearest centroids are within fp32 rounding (near-ties), and
+        # when they agree everywhere the centroids agree too
+        if torch.equal(klab, ref_h_lab):
+            assert torch.equal(kcent, ref_h_cent)
+        else:
+            tc = P.TieCounter()
+            for h in range(w.H):
+                x = P.np64(kr[0, h, :, d_t:d_t + d_h])
+                P.check_assign(x, P.np64(kcent[0, h]), klab[0, h].cpu().numpy(), tc, f"noalloc keys h{h}")
+            tc.assert_ok("noalloc keys")
 
 
 def test_noalloc_kmeans_512_clusters_against_oracle():
