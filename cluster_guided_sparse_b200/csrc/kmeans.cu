@@ -523,8 +523,7 @@ __global__ void __launch_bounds__(128) km_finalize_kernel(KmBatch b, int N)
     const int c = blockIdx.x, bh = blockIdx.y, d = threadIdx.x;
     if (c >= P.C) return;
     const int dn = P.dim_n;
-    const int32_t *start = P.start + (int64_t)bh * (P.C + 1);
-    const int sz = start[c + 1] - start[c];
+    const int sz = P.sizes[(int64_t)bh * P.C + c];
     const double scale = ldexp(1.0, fixed_shift(P.maxabs + bh, N));
     unsigned long long *sums = P.sums + ((int64_t)bh * P.C + c) * dn;
     float *cent = P.cent + ((int64_t)bh * P.C + c) * dn;

@@ -825,33 +825,43 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         return cls[item];
     };
     // Key walk without block-wide scans: warp w owns a contiguous chunk of the
-    // keys (a multiple of 64).  Pass 1 counts each chunk's keys above and at
-    // the cut; after one barrier every warp knows its chunk's output base, and
-    // pass 2 walks the chunk again, 64 keys per step (two per lane), placing
-    // each key by warp ballots.
+    // keys (a multiple of 256).  Each lane takes eight adjacent keys per step
+    // (one 16-byte load of their item ranks), so a warp step covers 256 keys.
+    // Pass 1 counts the chunk's keys above and at the cut in per-lane
+    // registers; after one barrier every warp knows its chunk's output base,
+    // and pass 2 walks the chunk again, placing each lane's keys after an
+    // exclusive warp scan of the lanes' counts.
     const uint16_t *ki = a.key_item + (int64_t)bh * a.N;
-    const bool pair = (((int64_t)bh * a.N) & 1) == 0;  // 4-byte aligned pairs of ranks
+    const bool vec8 = (((int64_t)bh * a.N) & 7) == 0;  // 16-byte aligned runs of eight ranks
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-    const int chunk = (((a.N + nwarps - 1) / nwarps) + 63) & ~63;
+    const int chunk = (((a.N + nwarps - 1) / nwarps) + 255) & ~255;
     const int j_begin = min(a.N, warp * chunk), j_end = min(a.N, j_begin + chunk);
     __shared__ int wgt[32], weq[32];
-    auto classes = [&](int j0, uint8_t &k0, uint8_t &k1) {
-        const int j = j0 + 2 * lane;
-        if (pair && j + 1 < j_end) {
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(ki + j);
-            k0 = class_of(w & 0xffffu);
-            k1 = class_of(w >> 16);
+    // classes of keys j .. j+7: 2 above the cut, 1 at it, 0 below (or past the chunk)
+    auto classes8 = [&](int j, uint8_t (&k)[8]) {
+        if (vec8 && j + 8 <= j_end) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(ki + j);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int t = 0; t < 8; ++t) k[t] = class_of((ws[t >> 1] >> (16 * (t & 1))) & 0xffffu);
         } else {
-            k0 = j < j_end ? class_of(ki[j]) : 0;
-            k1 = j + 1 < j_end ? class_of(ki[j + 1]) : 0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) k[t] = j + t < j_end ? class_of(ki[j + t]) : 0;
         }
     };
     int g_cnt = 0, e_cnt = 0;
-    for (int j0 = j_begin; j0 < j_end; j0 += 64) {
-        uint8_t k0, k1;
-        classes(j0, k0, k1);
-        g_cnt += __popc(__ballot_sync(0xffffffffu, k0 == 2)) + __popc(__ballot_sync(0xffffffffu, k1 == 2));
-        e_cnt += __popc(__ballot_sync(0xffffffffu, k0 == 1)) + __popc(__ballot_sync(0xffffffffu, k1 == 1));
+    for (int j0 = j_begin; j0 < j_end; j0 += 256) {
+        uint8_t k[8];
+        classes8(j0 + 8 * lane, k);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            g_cnt += k[t] == 2;
+            e_cnt += k[t] == 1;
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        g_cnt += __shfl_xor_sync(0xffffffffu, g_cnt, o);
+        e_cnt += __shfl_xor_sync(0xffffffffu, e_cnt, o);
     }
     if (lane == 0) {
         wgt[warp] = g_cnt;
@@ -863,24 +873,35 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         g += wgt[w];
         e += weq[w];
     }
-    const uint32_t lt = lanemask_lt();
-    for (int j0 = j_begin; j0 < j_end; j0 += 64) {
-        uint8_t k0, k1;
-        classes(j0, k0, k1);
-        const uint32_t g0 = __ballot_sync(0xffffffffu, k0 == 2), g1 = __ballot_sync(0xffffffffu, k1 == 2);
-        const uint32_t e0 = __ballot_sync(0xffffffffu, k0 == 1), e1 = __ballot_sync(0xffffffffu, k1 == 1);
-        // keys before this lane's first key: both keys of every lower lane
-        unsigned gl = g + __popc(g0 & lt) + __popc(g1 & lt), el = e + __popc(e0 & lt) + __popc(e1 & lt);
-        const int j = j0 + 2 * lane;
+    for (int j0 = j_begin; j0 < j_end; j0 += 256) {
+        const int j = j0 + 8 * lane;
+        uint8_t k[8];
+        classes8(j, k);
+        unsigned lg = 0, le = 0;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const uint8_t kt = t ? k1 : k0;
-            if (kt == 2) {
+        for (int t = 0; t < 8; ++t) {
+            lg += k[t] == 2;
+            le += k[t] == 1;
+        }
+        // exclusive scan of the lanes' (above, at) counts, packed in one word
+        const unsigned packed = lg | (le << 16);
+        unsigned incl = packed;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const unsigned tot = __shfl_sync(0xffffffffu, incl, 31);
+        const unsigned ex = incl - packed;
+        unsigned gl = g + (ex & 0xffffu), el = e + (ex >> 16);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            if (k[t] == 2) {
                 const unsigned slot = gl + (el < (unsigned)need ? el : (unsigned)need);
                 if (slot < (unsigned)n) out[slot] = j + t;
                 else set_error(a.err, kErrRange, 0x300 + c);
                 ++gl;
-            } else if (kt == 1) {
+            } else if (k[t] == 1) {
                 if (el < (unsigned)need) {
                     if (gl + el < (unsigned)n) out[gl + el] = j + t;
                     else set_error(a.err, kErrRange, 0x300 + c);
@@ -888,8 +909,8 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
                 ++el;
             }
         }
-        g += __popc(g0) + __popc(g1);
-        e += __popc(e0) + __popc(e1);
+        g += tot & 0xffffu;
+        e += tot >> 16;
     }
 }
 
