@@ -33,16 +33,25 @@ __device__ __forceinline__ unsigned long long dkey(double d)
 
 struct BisectShared {
     double c[2][128];
-    double part[2][16][64];
+    double sum[2][128];
     int hist[256];
     int tmp[33];
     unsigned long long prefix;
-    int below, need, bucket;
+    int below, need, bucket, eq;
 };
 
-// Selects the `k` smallest keys (delta asc, member index asc) among n keys:
-// returns the cut key and how many members at exactly that key are taken.
-__device__ void select_k(BisectShared &S, const double *delta, int n, int k, unsigned long long *cut, int *need)
+// A node's median cut: members with keys below `key` go to child 0, and of
+// the `eq` members at exactly `key` the first `need` in member order.
+struct Cut {
+    unsigned long long key;
+    int need, eq;
+};
+
+// Selects the `k` smallest of n ordered 64-bit keys (key(i), member index
+// asc): the cut key, how many keys equal it and how many of those are
+// taken.  Eight 8-bit radix passes.
+template <class Key>
+__device__ void radix_select(BisectShared &S, Key key, int n, int k, Cut &c)
 {
     if (threadIdx.x == 0) {
         S.prefix = 0ull;
@@ -57,79 +66,264 @@ __device__ void select_k(BisectShared &S, const double *delta, int n, int k, uns
         // A node's deltas share their leading bytes, so most keys fall in one
         // bucket: add per warp (one atomic per distinct bucket) instead of
         // per key, which would serialise on that bucket.
-        for (int i0 = 0; i0 < n; i0 += blockDim.x) {
-            const int i = i0 + threadIdx.x;
-            int b = -1;
-            if (i < n) {
-                const unsigned long long u = dkey(delta[i]);
-                if (hi >= 64 || (u >> hi) == (pre >> hi)) b = (int)((u >> shift) & 255ull);
+        const int step = 4 * blockDim.x;
+        for (int i0 = 0; i0 < n; i0 += step) {
+            unsigned long long u[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = i0 + e * blockDim.x + threadIdx.x;
+                u[e] = i < n ? key(i) : 0ull;
             }
-            const unsigned peers = __match_any_sync(0xffffffffu, b);
-            if (b >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&S.hist[b], __popc(peers));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = i0 + e * blockDim.x + threadIdx.x;
+                int b = -1;
+                if (i < n && (hi >= 64 || (u[e] >> hi) == (pre >> hi))) b = (int)((u[e] >> shift) & 255ull);
+                const unsigned peers = __match_any_sync(0xffffffffu, b);
+                if (b >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&S.hist[b], __popc(peers));
+            }
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
-            int acc = S.below, b = 0;
-            for (; b < 255; ++b) {
-                if (acc + S.hist[b] >= k) break;
-                acc += S.hist[b];
+        if (threadIdx.x < 32) {
+            // the first bucket b (< 255) where the running count reaches k,
+            // else 255: lane L scans buckets 8L..8L+7 from its exclusive prefix
+            const int lane = threadIdx.x;
+            int h[8], loc = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                h[e] = S.hist[lane * 8 + e];
+                loc += h[e];
             }
-            S.below = acc;
-            S.prefix = pre | ((unsigned long long)b << shift);
+            const int before = S.below + warp_incl_scan(loc) - loc;
+            const unsigned hit = __ballot_sync(0xffffffffu, before + loc >= k);
+            if (lane == (hit ? __ffs(hit) - 1 : 31)) {
+                int acc = before, b = lane * 8, cnt = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e, ++b) {
+                    cnt = h[e];
+                    if (b == 255 || acc + h[e] >= k) break;
+                    acc += h[e];
+                }
+                S.below = acc;
+                S.eq = cnt;
+                S.prefix = pre | ((unsigned long long)b << shift);
+            }
         }
         __syncthreads();
     }
-    *cut = S.prefix;
-    *need = k - S.below;
+    c.key = S.prefix;
+    c.need = k - S.below;
+    c.eq = S.eq;  // the last pass's bucket holds exactly the keys equal to the cut
 }
 
-// delta = ||x - c0||^2 - ||x - c1||^2 in fp64, dims in order.
-__device__ __forceinline__ double split_delta(const __nv_bfloat16 *x, const double *c0, const double *c1, int D)
+__device__ __forceinline__ void select_k(BisectShared &S, const double *delta, int n, int k, Cut &c)
+{
+    radix_select(S, [&](int i) { return dkey(delta[i]); }, n, k, c);
+}
+
+// The same selection for large nodes in fewer passes over the deltas:
+// min and max, a histogram of 4096 equal-width buckets of the delta value
+// (the bucket is a non-decreasing function of delta, so every key of an
+// earlier bucket is below every key of a later one), the bucket where the
+// running count reaches k, and the radix select among that bucket's keys
+// only, gathered in shared memory.  A bucket holding more than kCoarseCap
+// keys falls back to the radix select over all n.
+constexpr int kCoarse = 4096, kCoarseCap = 2048;
+struct CoarseShared {
+    int hist[kCoarse];
+    unsigned long long list[kCoarseCap];
+    double red[2][32];
+    double lo, scale;
+    int nlist, bucket, below;
+};
+
+__device__ void select_k_coarse(BisectShared &S, CoarseShared &C, const double *delta, int n, int k, Cut &c)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    double lo = INFINITY, hi = -INFINITY;
+    for (int i = tid; i < n; i += blockDim.x) {
+        const double d = delta[i];
+        lo = fmin(lo, d);
+        hi = fmax(hi, d);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (lane == 0) {
+        C.red[0][warp] = lo;
+        C.red[1][warp] = hi;
+    }
+    for (int b = tid; b < kCoarse; b += blockDim.x) C.hist[b] = 0;
+    __syncthreads();
+    if (tid == 0) {
+        double l = C.red[0][0], h = C.red[1][0];
+        for (int w = 1; w < nw; ++w) {
+            l = fmin(l, C.red[0][w]);
+            h = fmax(h, C.red[1][w]);
+        }
+        C.lo = l;
+        C.scale = h > l ? (double)kCoarse / (h - l) : 0.0;
+        C.nlist = 0;
+    }
+    __syncthreads();
+    const double l = C.lo, sc = C.scale;
+    auto bucket_of = [&](double d) { return min(kCoarse - 1, (int)((d - l) * sc)); };
+    for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+        const int i = i0 + tid;
+        const int b = i < n ? bucket_of(delta[i]) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, b);
+        if (b >= 0 && lane == __ffs(peers) - 1) atomicAdd(&C.hist[b], __popc(peers));
+    }
+    __syncthreads();
+    // the first bucket where the running count reaches k: thread t scans
+    // buckets [t*per, (t+1)*per) from its exclusive prefix
+    const int per = kCoarse / blockDim.x;  // blockDim divides 4096
+    int loc = 0;
+    for (int e = 0; e < per; ++e) loc += C.hist[tid * per + e];
+    int tot;
+    const int before = block_excl_scan(loc, S.tmp, tot);
+    if (before < k && before + loc >= k) {
+        int acc = before, b = tid * per;
+        for (; acc + C.hist[b] < k; ++b) acc += C.hist[b];
+        C.bucket = b;
+        C.below = acc;
+    }
+    __syncthreads();
+    const int bk = C.bucket, below = C.below, m = C.hist[bk];
+    if (m > kCoarseCap) {
+        select_k(S, delta, n, k, c);
+        return;
+    }
+    for (int i = tid; i < n; i += blockDim.x) {
+        const double d = delta[i];
+        if (bucket_of(d) == bk) C.list[atomicAdd(&C.nlist, 1)] = dkey(d);
+    }
+    __syncthreads();
+    radix_select(S, [&](int i) { return C.list[i]; }, m, k - below, c);
+}
+
+// delta = ||x - c0||^2 - ||x - c1||^2 in fp64, dims in order.  The row is
+// read 8 dims (16 bytes) at a time (rows are 16-byte aligned).
+template <int D>
+__device__ __forceinline__ double split_delta(const __nv_bfloat16 *x, const double *c0, const double *c1)
 {
     double d0 = 0.0, d1 = 0.0;
-    for (int k = 0; k < D; ++k) {
-        const double xv = (double)__bfloat162float(x[k]);
-        const double t0 = xv - c0[k], t1 = xv - c1[k];
-        d0 = fma(t0, t0, d0);
-        d1 = fma(t1, t1, d1);
+#pragma unroll 2
+    for (int k0 = 0; k0 < D; k0 += 8) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(x + k0);
+        const __nv_bfloat16 *xv8 = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double xv = (double)__bfloat162float(xv8[e]);
+            const double t0 = xv - c0[k0 + e], t1 = xv - c1[k0 + e];
+            d0 = fma(t0, t0, d0);
+            d1 = fma(t1, t1, d1);
+        }
     }
     return d0 - d1;
 }
 
-// One ordered pass over a node's members: f(i, side0) for every thread and
-// every block of members (i >= n gives side0 = false), where side0 says
-// member i goes to child 0 under (cut, need) -- keys below the cut, then the
-// first `need` members at the cut in member order.  Block-wide.
+// Member sides under a cut, block-wide: f(i, side0) once for every member
+// i < n, where side0 says member i goes to child 0.  Without ties at the cut
+// (every member at the cut is taken) that is a plain comparison; otherwise
+// the members are visited in tiles of blockDim in member order and a block
+// scan ranks the members at the cut.
 template <class F>
-__device__ void each_side(BisectShared &S, const double *delta, int n, unsigned long long cut, int need, F &&f)
+__device__ void mark_sides(BisectShared &S, const double *delta, int n, const Cut &c, F &&f)
 {
+    if (c.need == c.eq) {
+        for (int i = threadIdx.x; i < n; i += blockDim.x) f(i, dkey(delta[i]) <= c.key);
+        return;
+    }
     int eq_run = 0;
     for (int b0 = 0; b0 < n; b0 += blockDim.x) {
         const int i = b0 + threadIdx.x;
         const unsigned long long u = i < n ? dkey(delta[i]) : ~0ull;
-        const int eq = (i < n && u == cut) ? 1 : 0;
+        const int eq = (i < n && u == c.key) ? 1 : 0;
         int tot;
         const int ex = block_excl_scan(eq, S.tmp, tot);
-        f(i, i < n && (u < cut || (eq && eq_run + ex < need)));
+        if (i < n) f(i, u < c.key || (eq && eq_run + ex < c.need));
         eq_run += tot;
     }
 }
 
-// Stable partition of a node's members by side: child 0 in member order, then child 1.
-__device__ void partition_node(BisectShared &S, const double *delta, int n, unsigned long long cut, int need,
-                               const int32_t *mem, int32_t *out)
+// Stable partition of a node's members by side: child 0 in member order,
+// then child 1.  Tiles of 4 members per thread; one block scan per tile
+// places child 0 (a second one ranks the members at the cut when some of
+// them are left out).
+__device__ void partition_node(BisectShared &S, const double *delta, int n, const Cut &c, const int32_t *mem,
+                               int32_t *out)
 {
+    constexpr int E = 4;
     const int half = n >> 1;
-    int s0_run = 0;
-    each_side(S, delta, n, cut, need, [&](int i, bool side0) {
+    const bool ties = c.need != c.eq;
+    int s0_run = 0, eq_run = 0;
+    for (int b0 = 0; b0 < n; b0 += E * blockDim.x) {
+        const int i0 = b0 + threadIdx.x * E;
+        unsigned long long u[E];
+        int neq = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            u[e] = i0 + e < n ? dkey(delta[i0 + e]) : ~0ull;
+            neq += (i0 + e < n && u[e] == c.key) ? 1 : 0;
+        }
+        int eq_rank = 0;
+        if (ties) {
+            int tot;
+            eq_rank = eq_run + block_excl_scan(neq, S.tmp, tot);
+            eq_run += tot;
+        }
+        bool side0[E];
+        int ns0 = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const bool eq = i0 + e < n && u[e] == c.key;
+            side0[e] = i0 + e < n && (u[e] < c.key || (eq && (!ties || eq_rank < c.need)));
+            if (eq) ++eq_rank;
+            ns0 += side0[e] ? 1 : 0;
+        }
         int tot0;
-        const int ex0 = block_excl_scan(side0 ? 1 : 0, S.tmp, tot0);
-        if (i < n) {
-            const int pos0 = s0_run + ex0;
-            out[side0 ? pos0 : half + (i - pos0)] = mem[i];
+        int pos0 = s0_run + block_excl_scan(ns0, S.tmp, tot0);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int i = i0 + e;
+            if (i < n) {
+                if (side0[e]) out[pos0++] = mem[i];
+                else out[half + (i - pos0)] = mem[i];
+            }
         }
         s0_run += tot0;
-    });
+    }
+}
+
+// Adds member i's row into its side's sums, warp-wide: every lane holds
+// D/32 consecutive dims of both sides' running sums.  The sums of bf16
+// values in fp64 are exact, so the order of the additions does not matter.
+template <int D>
+__device__ __forceinline__ void add_row(const __nv_bfloat16 *x, bool side0, double (&s0)[D / 32], double (&s1)[D / 32])
+{
+    constexpr int PER = D / 32;
+    const int lane = threadIdx.x & 31;
+    float v[PER];
+    if constexpr (PER == 4) {
+        const uint2 raw = *reinterpret_cast<const uint2 *>(x + lane * 4);
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&raw.x);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&raw.y);
+        v[0] = __low2float(a);
+        v[1] = __high2float(a);
+        v[2] = __low2float(b);
+        v[3] = __high2float(b);
+    } else {
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(x + lane * 2);
+        v[0] = __low2float(a);
+        v[1] = __high2float(a);
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        if (side0) s0[e] += (double)v[e];
+        else s1[e] += (double)v[e];
+    }
 }
 
 }  // namespace
@@ -146,12 +340,14 @@ struct BisectArgs {
 };
 
 // One CTA per (node, bh) of this level: 2-means split of the node's members.
+template <int D>
 __global__ void __launch_bounds__(kBT) bisect_level_kernel(BisectArgs a)
 {
     __shared__ BisectShared S;
     const int node = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-    const int n = a.N >> a.level, D = a.D, half = n >> 1;
-    const int nsl = blockDim.x >> 6;  // member slices of the update (blockDim in 128..1024)
+    const int n = a.N >> a.level, half = n >> 1;
+    const int lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    constexpr int PER = D / 32;
     int32_t *mem = a.order + (int64_t)bh * a.N + (int64_t)node * n;
     int32_t *out = a.order_tmp + (int64_t)bh * a.N + (int64_t)node * n;
     double *delta = a.delta + (int64_t)bh * a.N + (int64_t)node * n;
@@ -162,48 +358,36 @@ __global__ void __launch_bounds__(kBT) bisect_level_kernel(BisectArgs a)
         S.c[which][dim] = (double)__bfloat162float(X[(int64_t)mem[which ? half : 0] * D + dim]);
     }
     __syncthreads();
-    unsigned long long cut = 0;
-    int need = 0;
+    Cut cut;
     for (int r = 0; r <= a.iters; ++r) {
         // delta of every member
-        for (int i = tid; i < n; i += blockDim.x) delta[i] = split_delta(X + (int64_t)mem[i] * D, S.c[0], S.c[1], D);
+        for (int i = tid; i < n; i += blockDim.x) delta[i] = split_delta<D>(X + (int64_t)mem[i] * D, S.c[0], S.c[1]);
         __syncthreads();
-        select_k(S, delta, n, half, &cut, &need);
+        select_k(S, delta, n, half, cut);
         if (r == a.iters) break;
         // mark sides, reusing delta as the side flag for the sums (a thread
         // reads and then overwrites only its own member's entry)
-        each_side(S, delta, n, cut, need, [&](int i, bool side0) {
-            if (i < n) delta[i] = side0 ? 0.0 : 1.0;
-        });
+        mark_sides(S, delta, n, cut, [&](int i, bool side0) { delta[i] = side0 ? 0.0 : 1.0; });
+        for (int k = tid; k < 2 * D; k += blockDim.x) S.sum[k / D][k % D] = 0.0;
         __syncthreads();
-        // update: exact fp64 sums of each side (64 dims x blockDim/64 member
-        // slices per pass; exact, so the slicing does not change the sums)
-        for (int d0 = 0; d0 < D; d0 += 64) {
-            const int dim = tid & 63, slice = tid >> 6;
-            double s0 = 0.0, s1 = 0.0;
-            if (d0 + dim < D) {
-                for (int i = slice; i < n; i += nsl) {
-                    const double xv = (double)__bfloat162float(X[(int64_t)mem[i] * D + d0 + dim]);
-                    if (delta[i] == 0.0) s0 += xv;
-                    else s1 += xv;
-                }
-            }
-            S.part[0][slice][dim] = s0;
-            S.part[1][slice][dim] = s1;
-            __syncthreads();
-            if (tid < 128) {
-                const int which = tid >> 6, dd = tid & 63;
-                if (d0 + dd < D) {
-                    double sum = 0.0;
-                    for (int q = 0; q < nsl; ++q) sum += S.part[which][q][dd];
-                    S.c[which][d0 + dd] = sum / (double)half;
-                }
-            }
-            __syncthreads();
+        // update: each warp adds whole rows into its registers, then the
+        // warps' sums meet in shared memory (exact, so in any order)
+        double s0[PER], s1[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) s0[e] = s1[e] = 0.0;
+#pragma unroll 4
+        for (int i = warp; i < n; i += nw) add_row<D>(X + (int64_t)mem[i] * D, delta[i] == 0.0, s0, s1);
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            atomicAdd(&S.sum[0][lane * PER + e], s0[e]);
+            atomicAdd(&S.sum[1][lane * PER + e], s1[e]);
         }
+        __syncthreads();
+        for (int k = tid; k < 2 * D; k += blockDim.x) S.c[k / D][k % D] = S.sum[k / D][k % D] / (double)half;
+        __syncthreads();
     }
     // stable partition by the final cut: side 0 (member order), then side 1
-    partition_node(S, delta, n, cut, need, mem, out);
+    partition_node(S, delta, n, cut, mem, out);
 }
 
 // ---------------------------------------------------------------- split levels
@@ -228,72 +412,74 @@ __global__ void __launch_bounds__(128) bis_init_kernel(BisectArgs a)
     }
 }
 
+template <int D>
 __global__ void __launch_bounds__(kSplitRows) bis_delta_kernel(BisectArgs a, int nodes)
 {
-    const int bh = blockIdx.y, D = a.D;
-    const int p = blockIdx.x * kSplitRows + threadIdx.x;
+    __shared__ double c[2 * D];
+    const int bh = blockIdx.y;
+    const int p0 = blockIdx.x * kSplitRows, p = p0 + threadIdx.x;
+    const int n = a.N >> a.level;  // n >= kSplitRows and n % kSplitRows == 0 on split levels
+    const double *cg = a.cent + ((int64_t)bh * nodes + p0 / n) * 2 * D;
+    for (int k = threadIdx.x; k < 2 * D; k += kSplitRows) c[k] = cg[k];
+    __syncthreads();
     if (p >= a.N) return;
-    const int n = a.N >> a.level, node = p / n;
     const int32_t m = a.order[(int64_t)bh * a.N + p];
-    const double *c = a.cent + ((int64_t)bh * nodes + node) * 2 * D;
-    a.delta[(int64_t)bh * a.N + p] = split_delta(a.X + ((int64_t)bh * a.N + m) * D, c, c + D, D);
+    a.delta[(int64_t)bh * a.N + p] = split_delta<D>(a.X + ((int64_t)bh * a.N + m) * D, c, c + D);
 }
 
 // last == 0: mark each member's child; last == 1: write the children.
 __global__ void __launch_bounds__(kBT) bis_select_kernel(BisectArgs a, int last)
 {
     __shared__ BisectShared S;
+    __shared__ CoarseShared C;
     const int node = blockIdx.x, bh = blockIdx.y;
     const int n = a.N >> a.level;
     const int64_t base = (int64_t)bh * a.N + (int64_t)node * n;
     const double *delta = a.delta + base;
-    unsigned long long cut = 0;
-    int need = 0;
-    select_k(S, delta, n, n >> 1, &cut, &need);
+    Cut cut;
+    select_k_coarse(S, C, delta, n, n >> 1, cut);
     if (last) {
-        partition_node(S, delta, n, cut, need, a.order + base, a.order_tmp + base);
+        partition_node(S, delta, n, cut, a.order + base, a.order_tmp + base);
     } else {
         uint8_t *side = a.side + base;
-        each_side(S, delta, n, cut, need, [&](int i, bool side0) {
-            if (i < n) side[i] = side0 ? 0 : 1;
-        });
+        mark_sides(S, delta, n, cut, [&](int i, bool side0) { side[i] = side0 ? 0 : 1; });
     }
 }
 
-// Side sums of kSplitRows consecutive members (all of one node): 64 dims x
-// kSplitRows/64 member slices per pass, then one fp64 atomic per (side, dim).
+// Side sums of kSplitRows consecutive members (all of one node): a warp takes
+// 32 members, adds their rows into its registers (add_row), the CTA's warps
+// meet in shared memory, and one fp64 atomic per (side, dim) adds the CTA's
+// sums to the node's.
+template <int D>
 __global__ void __launch_bounds__(kSplitRows) bis_sums_kernel(BisectArgs a, int nodes)
 {
-    __shared__ double part[2][kSplitRows / 64][64];
-    const int bh = blockIdx.y, D = a.D, tid = threadIdx.x;
+    __shared__ double sum[2][D];
+    constexpr int PER = D / 32;
+    const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int p0 = blockIdx.x * kSplitRows;
-    const int n = a.N >> a.level, node = p0 / n;
-    const int32_t *mem = a.order + (int64_t)bh * a.N;
-    const uint8_t *side = a.side + (int64_t)bh * a.N;
+    const int node = p0 / (a.N >> a.level);
+    for (int k = tid; k < 2 * D; k += kSplitRows) sum[k / D][k % D] = 0.0;
+    const int i = p0 + warp * 32 + lane;  // N is a multiple of kSplitRows here
+    const int mi = a.order[(int64_t)bh * a.N + i];
+    const int si = a.side[(int64_t)bh * a.N + i];
     const __nv_bfloat16 *X = a.X + (int64_t)bh * a.N * D;
-    double *g = a.gsum + ((int64_t)bh * nodes + node) * 2 * D;
-    const int dim = tid & 63, slice = tid >> 6;
-    for (int d0 = 0; d0 < D; d0 += 64) {
-        double s0 = 0.0, s1 = 0.0;
-        if (d0 + dim < D)
-            for (int i = p0 + slice; i < p0 + kSplitRows; i += kSplitRows / 64) {
-                const double xv = (double)__bfloat162float(X[(int64_t)mem[i] * D + d0 + dim]);
-                if (side[i] == 0) s0 += xv;
-                else s1 += xv;
-            }
-        part[0][slice][dim] = s0;
-        part[1][slice][dim] = s1;
-        __syncthreads();
-        if (tid < 128) {
-            const int which = tid >> 6, dd = tid & 63;
-            if (d0 + dd < D) {
-                double sum = 0.0;
-                for (int q = 0; q < kSplitRows / 64; ++q) sum += part[which][q][dd];
-                atomicAdd(g + which * D + d0 + dd, sum);
-            }
-        }
-        __syncthreads();
+    double s0[PER], s1[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) s0[e] = s1[e] = 0.0;
+#pragma unroll 8
+    for (int r = 0; r < 32; ++r) {
+        const int m = __shfl_sync(0xffffffffu, mi, r), sd = __shfl_sync(0xffffffffu, si, r);
+        add_row<D>(X + (int64_t)m * D, sd == 0, s0, s1);
     }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        atomicAdd(&sum[0][lane * PER + e], s0[e]);
+        atomicAdd(&sum[1][lane * PER + e], s1[e]);
+    }
+    __syncthreads();
+    double *g = a.gsum + ((int64_t)bh * nodes + node) * 2 * D;
+    for (int k = tid; k < 2 * D; k += kSplitRows) atomicAdd(g + k, sum[k / D][k % D]);
 }
 
 __global__ void __launch_bounds__(256) bis_means_kernel(BisectArgs a)
@@ -388,11 +574,13 @@ void launch_bisect(const __nv_bfloat16 *X, int BH, int N, int D, int leaf, int i
             bis_init_kernel<<<per_node, 128, 0, st>>>(a);
             count_launches(1);
             for (int r = 0; r <= iters; ++r) {
-                bis_delta_kernel<<<rows, kSplitRows, 0, st>>>(a, nodes);
+                if (D == 64) bis_delta_kernel<64><<<rows, kSplitRows, 0, st>>>(a, nodes);
+                else bis_delta_kernel<128><<<rows, kSplitRows, 0, st>>>(a, nodes);
                 bis_select_kernel<<<per_node, kBT, 0, st>>>(a, r == iters ? 1 : 0);
                 count_launches(2);
                 if (r == iters) break;
-                bis_sums_kernel<<<rows, kSplitRows, 0, st>>>(a, nodes);
+                if (D == 64) bis_sums_kernel<64><<<rows, kSplitRows, 0, st>>>(a, nodes);
+                else bis_sums_kernel<128><<<rows, kSplitRows, 0, st>>>(a, nodes);
                 bis_means_kernel<<<per_node, 256, 0, st>>>(a);
                 count_launches(2);
             }
@@ -400,7 +588,8 @@ void launch_bisect(const __nv_bfloat16 *X, int BH, int N, int D, int leaf, int i
             // a CTA as wide as its node (128..1024 threads): deep levels have many
             // small nodes, and idle threads would only wait at the barriers
             const int threads = n >= kBT ? kBT : (n > 128 ? (n + 63) & ~63 : 128);
-            bisect_level_kernel<<<dim3(nodes, BH), threads, 0, st>>>(a);
+            if (D == 64) bisect_level_kernel<64><<<dim3(nodes, BH), threads, 0, st>>>(a);
+            else bisect_level_kernel<128><<<dim3(nodes, BH), threads, 0, st>>>(a);
             count_launches(1);
         }
         int32_t *t = cur;

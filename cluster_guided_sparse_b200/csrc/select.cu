@@ -39,29 +39,59 @@ struct SelArgs {
 
 // -------------------------------------------------------------- LUT
 // lut[c][e] for e over (t: 0..Ct-1, h: Ct.., w: Ct+Ch..): fp64 dot of the
-// query centroid's subspace slice with the key centroid, stored as fp32.
-__global__ void lut_kernel(const float *qcent, const float *kc_t, const float *kc_h, const float *kc_w,
-                           float *lut, int Cq, int D, int dt, int dh, int dw, int Ct, int Ch, int Cw)
+// query centroid's subspace slice with the key centroid, summed in dimension
+// order, stored as fp32.  A CTA takes kLutQ query centroids of one head and
+// walks the key centroids of each subspace in tiles of kLutRows rows, each
+// tile staged in shared memory by coalesced loads (rows padded to an odd
+// stride, so the row-per-lane reads are conflict-free); a thread owns one
+// row and kLutQ / kLutGroups of the query centroids.
+constexpr int kLutQ = 16, kLutRows = 64, kLutGroups = 4, kLutThreads = kLutRows * kLutGroups;
+
+__global__ void __launch_bounds__(kLutThreads)
+    lut_kernel(const float *qcent, const float *kc_t, const float *kc_h, const float *kc_w, float *lut, int Cq, int D,
+               int dt, int dh, int dw, int Ct, int Ch, int Cw)
 {
-    extern __shared__ float q[];
-    const int c = blockIdx.x, bh = blockIdx.y;
-    const float *qc = qcent + ((int64_t)bh * Cq + c) * D;
-    for (int k = threadIdx.x; k < D; k += blockDim.x) q[k] = qc[k];
-    __syncthreads();
+    extern __shared__ float lsm[];
+    constexpr int QPT = kLutQ / kLutGroups;  // query centroids per thread
+    const int c0 = blockIdx.x * kLutQ, bh = blockIdx.y;
+    const int nq = min(kLutQ, Cq - c0);
+    float *q = lsm;                  // [kLutQ][D]
+    float *kt = lsm + kLutQ * D;     // [kLutRows][stride]
+    for (int i = threadIdx.x; i < kLutQ * D; i += kLutThreads)
+        q[i] = i / D < nq ? qcent[((int64_t)bh * Cq + c0) * D + i] : 0.f;
     const int Csum = Ct + Ch + Cw;
-    for (int e = threadIdx.x; e < Csum; e += blockDim.x) {
-        const float *kc;
-        int off, ds;
-        if (e < Ct) {
-            kc = kc_t + ((int64_t)bh * Ct + e) * dt; off = 0; ds = dt;
-        } else if (e < Ct + Ch) {
-            kc = kc_h + ((int64_t)bh * Ch + (e - Ct)) * dh; off = dt; ds = dh;
-        } else {
-            kc = kc_w + ((int64_t)bh * Cw + (e - Ct - Ch)) * dw; off = dt + dh; ds = dw;
+    const int row = threadIdx.x % kLutRows, grp = threadIdx.x / kLutRows;
+    const float *segs[3] = {kc_t, kc_h, kc_w};
+    const int dss[3] = {dt, dh, dw}, Cs[3] = {Ct, Ch, Cw}, offs[3] = {0, dt, dt + dh};
+    int col = 0;
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        const int ds = dss[s], stride = ds | 1;
+        for (int e0 = 0; e0 < Cs[s]; e0 += kLutRows) {
+            const int rows = min(kLutRows, Cs[s] - e0);
+            __syncthreads();  // q staged / previous tile consumed
+            const float *src = segs[s] + ((int64_t)bh * Cs[s] + e0) * ds;
+            for (int i = threadIdx.x; i < rows * ds; i += kLutThreads) kt[(i / ds) * stride + i % ds] = src[i];
+            __syncthreads();
+            if (row < rows) {
+                double acc[QPT];
+#pragma unroll
+                for (int u = 0; u < QPT; ++u) acc[u] = 0.0;
+                const float *kr = kt + row * stride;
+                const float *qs = q + grp * QPT * D + offs[s];
+                for (int k = 0; k < ds; ++k) {
+                    const double kv = (double)kr[k];
+#pragma unroll
+                    for (int u = 0; u < QPT; ++u) acc[u] += (double)qs[u * D + k] * kv;
+                }
+#pragma unroll
+                for (int u = 0; u < QPT; ++u) {
+                    const int c = grp * QPT + u;
+                    if (c < nq) lut[((int64_t)bh * Cq + c0 + c) * Csum + col + e0 + row] = (float)acc[u];
+                }
+            }
         }
-        double s = 0.0;
-        for (int k = 0; k < ds; ++k) s += (double)q[off + k] * (double)kc[k];
-        lut[((int64_t)bh * Cq + c) * Csum + e] = (float)s;
+        col += Cs[s];
     }
 }
 
@@ -938,8 +968,10 @@ cudaError_t select_configure()
 void launch_lut(const float *qcent, const float *kc_t, const float *kc_h, const float *kc_w, float *lut, int BH,
                 int Cq, int D, int dt, int dh, int dw, int Ct, int Ch, int Cw, cudaStream_t st)
 {
-    lut_kernel<<<dim3(Cq, BH), 128, D * sizeof(float), st>>>(qcent, kc_t, kc_h, kc_w, lut, Cq, D, dt, dh, dw, Ct,
-                                                            Ch, Cw);
+    const int dmax = max(dt, max(dh, dw));
+    const size_t smem = ((size_t)kLutQ * D + (size_t)kLutRows * (dmax | 1)) * sizeof(float);
+    lut_kernel<<<dim3((Cq + kLutQ - 1) / kLutQ, BH), kLutThreads, smem, st>>>(qcent, kc_t, kc_h, kc_w, lut, Cq, D, dt,
+                                                                             dh, dw, Ct, Ch, Cw);
     count_launches(1);
 }
 

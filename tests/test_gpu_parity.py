@@ -247,9 +247,16 @@ def test_degenerate_identical_tokens_leave_clusters_empty():
                                atol=2e-2)
 
 
-def bisect_parity(w, heads, cl_sample=None, q_sample=None, seed=0):
+def bisect_parity(w, heads, cl_sample=None, q_sample=None, seed=0, tie_groups=0):
     rng = np.random.default_rng(seed)
     q, k, v = synth.make_inputs(w)
+    if tie_groups:
+        # 90% of the rows become copies of `tie_groups` rows, so the median
+        # cuts fall among equal deltas (member-order tie rule)
+        idx = torch.from_numpy(np.nonzero(rng.random(w.N) < 0.9)[0])
+        src = torch.from_numpy(rng.integers(0, w.N, tie_groups))[idx % tie_groups]
+        for t in (q, k):
+            t[:, :, idx] = t[:, :, src]
     qd, kd, vd = to_dev(q, k, v)
     pl = plan_of(w, qd, kd)
     o = scope.attn(qd, kd, vd, pl)
@@ -295,6 +302,13 @@ def test_bisection_small_shapes(N, D, H):
     w = synth.WORKLOADS["unstructured"].with_(N=N, D=D, H=H, d_split=(D, 0, 0), components=16, k_min=32,
                                                config_id=150 + N, c_q=N // 64, c_sub=(N // 64, 1, 1))
     bisect_parity(w, range(H))
+
+
+@pytest.mark.parametrize("groups", [1, 3, 24])
+def test_bisection_tied_rows(groups):
+    w = synth.WORKLOADS["unstructured"].with_(N=4096, D=64, H=1, d_split=(64, 0, 0), components=16, k_min=32,
+                                               config_id=170 + groups, c_q=64, c_sub=(64, 1, 1))
+    bisect_parity(w, [0], tie_groups=groups)
 
 
 # ClusterAttention compensation: every excluded key enters through its key
