@@ -26,7 +26,8 @@ SCOPE_F32, SCOPE_BF16, SCOPE_I32, SCOPE_I64 = 0, 1, 2, 3
 STATUS = {0: "SCOPE_OK", 1: "SCOPE_EINVAL", 2: "SCOPE_ESHAPE", 3: "SCOPE_EDTYPE", 4: "SCOPE_EALIGN",
           5: "SCOPE_EWORKSPACE", 6: "SCOPE_ECAPACITY", 7: "SCOPE_ECUDA", 8: "SCOPE_ETIMEOUT", 9: "SCOPE_EDEVICE"}
 VIEWS = ["qr", "kr", "q_labels", "q_centroids", "q_sizes", "q_perm", "q_start", "k_codes", "k_cent_t",
-         "k_cent_h", "k_cent_w", "lut", "r", "kh", "n", "offsets", "indices", "error", "eg_entropy", "eg_pool", "fixup"]
+         "k_cent_h", "k_cent_w", "lut", "r", "kh", "n", "offsets", "indices", "error", "eg_entropy", "eg_pool", "fixup",
+         "group_indices", "group_n", "group_masks"]
 _TORCH_DT = {SCOPE_F32: torch.float32, SCOPE_BF16: torch.bfloat16, SCOPE_I32: torch.int32, SCOPE_I64: torch.int64}
 
 

@@ -67,11 +67,18 @@ struct Args {
     const int32_t *n_c;        // [BH][Cq] or null
     int32_t *err;
     float *lse;                // [BH][N] natural log-sum-exp of every stored row, or null
+    // Grouped work items (ClusterAttention leaves of 32 or 64 queries): item =
+    // (bh, group of L consecutive leaves), `indices` holds the groups' union
+    // lists at their first leaf's offset, u_n their lengths, and gmask the
+    // per-tile, per-leaf 128-bit membership masks (null: one cluster per item).
+    const uint32_t *gmask;
+    const int32_t *u_n;
+    int L, leaf_shift, G;
     int N, Cq;
     float scale_log2;          // log2(e) / sqrt(D)
 };
 
-template <int D>
+template <int D, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(Args a)
 {
@@ -91,16 +98,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int item = blockIdx.x;
-    if (item >= *a.n_items) return;  // uniform for the CTA
-    const int4 it = a.items[item];
-    const int bh = it.x, c = it.y, q0 = it.z, nq = it.w;
+    int bh, c, q0, nq, grp = 0;
+    if constexpr (GROUPED) {  // grid = BH * G: one item per (bh, group), all 256 rows
+        bh = item / a.G;
+        grp = item % a.G;
+        c = grp * a.L;
+        q0 = 0;
+        nq = a.L << a.leaf_shift;
+    } else {
+        if (item >= *a.n_items) return;  // uniform for the CTA
+        const int4 it = a.items[item];
+        bh = it.x;
+        c = it.y;
+        q0 = it.z;
+        nq = it.w;
+    }
     const bool two = nq > BM;
     const int64_t base = (int64_t)bh * a.N;
     const __nv_bfloat16 *vbh = a.v + a.vs.bh_off(bh);
     const int64_t vsn = a.vs.sN;
     const int cstart = a.start ? a.start[(int64_t)bh * (a.Cq + 1) + c] : 0;
     const long long loff = a.indices ? a.offsets[(int64_t)bh * a.Cq + c] : 0;
-    const int nk = a.indices ? a.n_c[(int64_t)bh * a.Cq + c] : a.N;
+    const int nk = GROUPED ? a.u_n[(int64_t)bh * a.G + grp] : a.indices ? a.n_c[(int64_t)bh * a.Cq + c] : a.N;
+    // first mask slot of the group (kept disjoint across groups by the +item)
+    const long long mslot = GROUPED ? loff / 128 + item : 0;
+    if (GROUPED && nk <= 0) return;  // uniform; a group's leaves always hold keys
     const int ntiles = (nk + BN - 1) / BN;
 
     if (threadIdx.x == 0) {
@@ -266,7 +288,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool active = t == 0 || two;
         float m_run = -INFINITY, l = 0.f;
         bool ok = active;
+        // grouped items: this row's leaf inside the group and its mask words
+        const uint4 *gm = GROUPED ? reinterpret_cast<const uint4 *>(a.gmask) + mslot * a.L +
+                                        ((t * BM + row) >> a.leaf_shift)
+                                  : nullptr;
         for (int j = 0; ok && j < ntiles; ++j) {
+            uint4 mw;
+            if constexpr (GROUPED) mw = __ldg(gm + (int64_t)j * a.L);  // in flight during the wait
             if (!mbar_wait(&bar_s_full[t], j & 1, abort_flag, a.err, 0x30 + t)) {
                 ok = false;
                 break;
@@ -281,6 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < BN; ++i)
                     if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+            }
+            if constexpr (GROUPED) {
+                if ((mw.x & mw.y & mw.z & mw.w) != ~0u) {  // warp-uniform: a warp's rows share a leaf
+                    const uint32_t m4[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+                    for (int i = 0; i < BN; ++i)
+                        if (!((m4[i >> 5] >> (i & 31)) & 1u)) r[i] = __float_as_uint(-INFINITY);
+                }
             }
             // row max: three-input max, two new values per instruction, four chains
             float m4[4];
@@ -300,14 +336,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_run = mt;
             } else if (__any_sync(0xffffffffu, mt > m_run + 8.f)) {
                 const float mn = fmaxf(m_run, mt);
-                alpha = ex2(m_run - mn);
+                // grouped: a row with no key yet (m = -inf: every key so far
+                // masked) has l = 0 and O = 0, and takes alpha = 0
+                alpha = (GROUPED && m_run == -INFINITY) ? 0.f : ex2(m_run - mn);
                 m_run = mn;
                 l *= alpha;
                 rescale = true;
             }
             // p = 2^(s*scale - m) on pairs straight from the loaded row; row sum
-            // in four partial lanes; bf16 pairs written over S.
-            const uint64_t scp = f2pack(a.scale_log2, a.scale_log2), nmp = f2pack(-m_run, -m_run);
+            // in four partial lanes; bf16 pairs written over S.  (Grouped: while
+            // m is still -inf every p is 0; a finite reference keeps it so.)
+            const float m_ref = (GROUPED && m_run == -INFINITY) ? 0.f : m_run;
+            const uint64_t scp = f2pack(a.scale_log2, a.scale_log2), nmp = f2pack(-m_ref, -m_ref);
             uint64_t sA = 0ull, sB = 0ull;  // (0.f, 0.f)
 #pragma unroll
             for (int c4 = 0; c4 < BN / 32; ++c4) {
@@ -421,11 +461,18 @@ constexpr size_t tc_smem_bytes(int D)
 
 cudaError_t attn_tc_configure()
 {
-    cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tc_smem_bytes(128));
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(tc::attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)tc_smem_bytes(64));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::attn_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc_smem_bytes(64));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::attn_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc_smem_bytes(128));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::attn_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc_smem_bytes(64));
+    return e;
 }
 
 int attn_tc_max_items(int BH, int N, int Cq) { return BH * ((N + 2 * tc::BM - 1) / (2 * tc::BM) + Cq); }
@@ -456,10 +503,15 @@ bool rows_tensor_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int
 bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv_bfloat16 *v, const RowStrides &vs,
                     __nv_bfloat16 *o, const RowStrides &os, int4 *items, int32_t *n_items, int max_items, const int32_t *sizes, const int32_t *perm,
                     const int32_t *start, const long long *offsets, const int32_t *indices, const int32_t *n_c,
-                    int32_t *err, float *lse, int BH, int N, int D, int Cq, cudaStream_t st)
+                    int32_t *err, float *lse, int BH, int N, int D, int Cq, cudaStream_t st,
+                    const GroupedLists *grouped)
 {
-    tc::tc_items_kernel<<<1, 1024, 0, st>>>(sizes, items, n_items, BH, sizes ? Cq : 1, N);
-    count_launches(1);
+    if (grouped) {
+        max_items = BH * (Cq / grouped->L);
+    } else {
+        tc::tc_items_kernel<<<1, 1024, 0, st>>>(sizes, items, n_items, BH, sizes ? Cq : 1, N);
+        count_launches(1);
+    }
     tc::Args a;
     a.qr = qr;
     a.kr = kr;
@@ -476,13 +528,23 @@ bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv
     a.n_c = n_c;
     a.err = err;
     a.lse = lse;
+    a.gmask = grouped ? grouped->masks : nullptr;
+    a.u_n = grouped ? grouped->u_n : nullptr;
+    a.L = grouped ? grouped->L : 0;
+    a.leaf_shift = grouped ? grouped->leaf_shift : 0;
+    a.G = grouped ? Cq / grouped->L : 0;
+    if (grouped) a.indices = grouped->u_idx;
     a.N = N;
     a.Cq = Cq;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-    if (D == 128)
-        tc::attn_tc_kernel<128><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(a);
+    if (D == 128 && grouped)
+        tc::attn_tc_kernel<128, true><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(a);
+    else if (D == 128)
+        tc::attn_tc_kernel<128, false><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(a);
+    else if (grouped)
+        tc::attn_tc_kernel<64, true><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(a);
     else
-        tc::attn_tc_kernel<64><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(a);
+        tc::attn_tc_kernel<64, false><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(a);
     count_launches(1);
     return true;
 }

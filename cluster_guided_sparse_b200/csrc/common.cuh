@@ -38,6 +38,15 @@ struct KmProblem {
 // Where the rows of a caller's [B, H, N, D] tensor live: row (b, h, n)
 // starts at element b*sB + h*sH + n*sN (D contiguous elements).  Kernels index
 // by the flat (batch, head) number bh = b*H + h.
+// Grouped attention lists: L consecutive ClusterAttention leaves of 2^leaf_shift
+// queries share one work item over the union of their lists (pack.cu).
+struct GroupedLists {
+    const int32_t *u_idx;    // union lists at their group's first-leaf offset
+    const int32_t *u_n;      // [BH][Cq / L] union lengths
+    const uint32_t *masks;   // per tile and leaf, 128-bit membership masks
+    int L, leaf_shift;
+};
+
 struct RowStrides {
     int64_t sB, sH, sN;
     int H;

@@ -44,7 +44,10 @@ int attn_tc_max_items(int BH, int N, int Cq);
 bool launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, const RowStrides &,
                     __nv_bfloat16 *, const RowStrides &, int4 *, int32_t *, int, const int32_t *, const int32_t *,
                     const int32_t *, const long long *, const int32_t *, const int32_t *, int32_t *, float *, int, int,
-                    int, int, cudaStream_t);
+                    int, int, cudaStream_t, const GroupedLists *);
+size_t pack_mask_bytes(int64_t cap, int BH, int G, int L);
+void launch_pack_lists(const long long *, const int32_t *, const int32_t *, int32_t *, int32_t *, uint32_t *, int, int,
+                       int, int, cudaStream_t);
 void launch_compensate(const __nv_bfloat16 *, const __nv_bfloat16 *, const RowStrides &, const int32_t *,
                        const int32_t *, const int32_t *, const int32_t *, const int32_t *, const int32_t *,
                        const float *, float *, const long long *, const int32_t *, const int32_t *, const float *,
@@ -100,6 +103,8 @@ struct Layout {
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3], k_tsum[3];
     size_t sel_state, eg_state, lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
     size_t bis_order, bis_delta, bis_aux, q_chi, q_clo, q_sums, k_sums[3], sums_bytes, lse, vmean;
+    size_t u_idx, u_n, gmask;  // grouped attention lists (gL > 0)
+    int gL, gshift, G;         // leaves per group, log2(leaf), groups per head
     bool comp, eg, blocks;
     size_t total;
 };
@@ -393,6 +398,20 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.nwork = take(cur, 16);
     L.vb = take(cur, L.f32 ? BH * N * D * 2 : 0);
     L.indices = take(cur, (size_t)L.cap * 4);
+    // ClusterAttention leaves of 32 or 64 queries: 256 / leaf consecutive
+    // leaves share one attention work item over the union of their lists
+    L.gL = 0;
+    if (L.bisect && (p->fixed_cluster_size == 32 || p->fixed_cluster_size == 64)) {
+        const int gl = 256 / p->fixed_cluster_size;
+        if (L.Cq % gl == 0) {
+            L.gL = gl;
+            L.gshift = p->fixed_cluster_size == 32 ? 5 : 6;
+            L.G = L.Cq / gl;
+        }
+    }
+    L.u_idx = take(cur, L.gL ? (size_t)L.cap * 4 : 0);
+    L.u_n = take(cur, L.gL ? (size_t)BH * L.G * 4 : 0);
+    L.gmask = take(cur, L.gL ? pack_mask_bytes(L.cap, (int)BH, L.G, L.gL) : 0);
     L.total = cur;
     return L;
 }
@@ -635,6 +654,10 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
                   at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.r), at<int32_t>(ws, L.n), at<int32_t>(ws, L.kh),
                   at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), p->online_topk, ws + L.sel_state, (int)L.B,
                   p->eg_tau, p->eg_group, L.eg ? ws + L.eg_state : nullptr, L.blocks ? 1 : 0, s);
+    if (L.gL)
+        launch_pack_lists(at<long long>(ws, L.offsets), at<int32_t>(ws, L.n), at<int32_t>(ws, L.indices),
+                          at<int32_t>(ws, L.u_idx), at<int32_t>(ws, L.u_n), at<uint32_t>(ws, L.gmask), (int)BH, L.Cq,
+                          L.gL, (int)N, s);
     if ((st = launch_status("selection")) != SCOPE_OK) return st;
 
     scope_plan_s *h = (scope_plan_s *)malloc(sizeof(scope_plan_s));
@@ -693,11 +716,14 @@ extern "C" scope_status scope_attn(const scope_tensor *q, const scope_tensor *k,
     RowStrides vs;
     const __nv_bfloat16 *vb = v_bf16(L, ws, v, &vs, s);
     const RowStrides os = rows_of(o);
+    const GroupedLists grouped{at<int32_t>(ws, L.u_idx), at<int32_t>(ws, L.u_n), at<uint32_t>(ws, L.gmask), L.gL,
+                               L.gshift};
     if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, vs, (__nv_bfloat16 *)o->ptr, os,
                    at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, at<int32_t>(ws, L.q_sizes),
                    at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start), at<long long>(ws, L.offsets),
                    at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n), at<int32_t>(ws, L.stats) + 4,
-                   L.comp ? at<float>(ws, L.lse) : nullptr, (int)L.BH, (int)L.N, (int)L.D, L.Cq, s))
+                   L.comp ? at<float>(ws, L.lse) : nullptr, (int)L.BH, (int)L.N, (int)L.D, L.Cq, s,
+                   L.gL ? &grouped : nullptr))
         return fail(SCOPE_ECUDA, "scope_attn: tensor map encoding failed");
     if (L.comp)
         // ClusterAttention: excluded key clusters enter through their mean key and value
@@ -784,7 +810,7 @@ extern "C" scope_status scope_dense_attn(const scope_tensor *q, const scope_tens
     if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, vs, (__nv_bfloat16 *)o->ptr,
                         rows_of(o), at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, nullptr, nullptr, nullptr,
                         nullptr, nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, nullptr, (int)L.BH, (int)L.N,
-                        (int)L.D, 1, s))
+                        (int)L.D, 1, s, nullptr))
         return fail(SCOPE_ECUDA, "scope_dense_attn: tensor map encoding failed");
     return launch_status("scope_dense_attn");
 }
@@ -823,6 +849,18 @@ extern "C" scope_status scope_plan_view(const scope_plan_t *plan, int which, sco
     case SCOPE_VIEW_INDICES: set(L.indices, SCOPE_I32, 1, L.cap, 0, 0, 0); break;
     case SCOPE_VIEW_ERROR: set(L.stats + 16, SCOPE_I32, 1, 4, 0, 0, 0); break;
     case SCOPE_VIEW_FIXUP: set(L.fix, SCOPE_I32, 1, 1, 0, 0, 0); break;
+    case SCOPE_VIEW_GROUP_INDICES:
+        if (!L.gL) return fail(SCOPE_EINVAL, "view: the plan has no grouped lists");
+        set(L.u_idx, SCOPE_I32, 1, L.cap, 0, 0, 0);
+        break;
+    case SCOPE_VIEW_GROUP_N:
+        if (!L.gL) return fail(SCOPE_EINVAL, "view: the plan has no grouped lists");
+        set(L.u_n, SCOPE_I32, 3, B, H, L.G, 0);
+        break;
+    case SCOPE_VIEW_GROUP_MASKS:
+        if (!L.gL) return fail(SCOPE_EINVAL, "view: the plan has no grouped lists");
+        set(L.gmask, SCOPE_I32, 1, (int64_t)(pack_mask_bytes(L.cap, (int)L.BH, L.G, L.gL) / 4), 0, 0, 0);
+        break;
     case SCOPE_VIEW_EG_ENTROPY:
         if (!L.eg) return fail(SCOPE_EINVAL, "no EG-Sparse routing in this plan (eg_tau = 0)");
         set(L.eg_state, SCOPE_F32, 2, B, H, 0, 0);

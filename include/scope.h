@@ -226,7 +226,16 @@ typedef enum {
     SCOPE_VIEW_EG_ENTROPY = 18, /* f32  [B,H] EG-Sparse head entropy (eg_tau > 0) */
     SCOPE_VIEW_EG_POOL = 19,    /* i32  [B,H] pool (group) of a routed head, -1 if not routed */
     SCOPE_VIEW_FIXUP = 20,      /* i32  [1] rows the last tensor-core query assignment sent to the fp64 re-check */
-    SCOPE_VIEW_COUNT = 21
+    /* ClusterAttention leaves of 32 or 64 queries: L = 256 / leaf consecutive
+     * leaves form a group that the attention serves as one work item. */
+    SCOPE_VIEW_GROUP_INDICES = 21, /* i32 [capacity] ascending union of a group's lists, at the
+                                      OFFSETS entry of its first leaf */
+    SCOPE_VIEW_GROUP_N = 22,    /* i32  [B,H,c_q/L] union lengths          */
+    SCOPE_VIEW_GROUP_MASKS = 23, /* u32 words: for union tile t (128 keys) of group g of flat
+                                    head bh and leaf l of the group, 4 words at
+                                    ((OFFSETS[first leaf] / 128 + bh*c_q/L + g + t) * L + l) * 4;
+                                    bit i = key i of the tile is in leaf l's list */
+    SCOPE_VIEW_COUNT = 24
 } scope_view_id;
 
 typedef struct {

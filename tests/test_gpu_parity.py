@@ -247,6 +247,38 @@ def test_degenerate_identical_tokens_leave_clusters_empty():
                                atol=2e-2)
 
 
+def check_groups(pl, w, h, get, groups=None):
+    """Grouped attention lists (leaves of 32 or 64 queries): every group's
+    union is the ascending union of its leaves' lists, stored at its first
+    leaf's offset, and its tile masks mark exactly each leaf's own keys."""
+    leaf, C = w.fixed_cluster_size, w.N // w.fixed_cluster_size
+    Lg = 256 // leaf if leaf in (32, 64) else 0
+    if not Lg or C % Lg:
+        with pytest.raises(scope.ScopeError):
+            pl.view("group_n")
+        return 0
+    G = C // Lg
+    off = pl.view("offsets").cpu().numpy()
+    gidx = pl.view("group_indices")
+    gn = pl.view("group_n")[0, h].cpu().numpy()
+    gm = pl.view("group_masks")
+    for g in (range(G) if groups is None else groups):
+        lists = [get(c) for c in range(g * Lg, (g + 1) * Lg)]
+        u = np.unique(np.concatenate(lists))
+        start = int(off[h * C + g * Lg])
+        assert int(gn[g]) == len(u), (h, g)
+        assert (gidx[start:start + len(u)].cpu().numpy() == u).all(), (h, g)
+        T = (len(u) + 127) // 128
+        slot = start // 128 + h * G + g
+        words = gm[slot * Lg * 4:(slot + T) * Lg * 4].cpu().numpy().view(np.uint32).reshape(T, Lg, 4)
+        for li, lst in enumerate(lists):
+            bits = np.zeros(T * 128, dtype=np.uint8)
+            bits[:len(u)] = np.isin(u, lst)
+            want = np.packbits(bits.reshape(T * 4, 32), axis=1, bitorder="little").view("<u4").reshape(T, 4)
+            assert (words[:, li, :] == want).all(), (h, g, li)
+    return G
+
+
 def bisect_parity(w, heads, cl_sample=None, q_sample=None, seed=0, tie_groups=0):
     rng = np.random.default_rng(seed)
     q, k, v = synth.make_inputs(w)
@@ -289,6 +321,8 @@ def bisect_parity(w, heads, cl_sample=None, q_sample=None, seed=0, tie_groups=0)
                           pl.view("n")[0, h].cpu().numpy(), get, wq, N, D, clusters, tc)
         rows = np.arange(N) if q_sample is None else np.sort(rng.choice(N, q_sample, replace=False))
         P.check_attention(qr, kr, v[0, h].double().numpy(), qlab, get, P.np64(o[0, h]), rows)
+        ng = C // (256 // leaf) if leaf in (32, 64) and C % (256 // leaf) == 0 else 0
+        check_groups(pl, w, h, get, None if cl_sample is None or ng == 0 else rng.choice(ng, 16, replace=False))
     tc.assert_ok("bisection Top-p counts")
 
 
@@ -297,10 +331,12 @@ def test_unstructured_bisection_parity():
     bisect_parity(w, [0, w.H - 1], cl_sample=8, q_sample=48)
 
 
-@pytest.mark.parametrize("N,D,H", [(128, 64, 1), (512, 128, 2), (4096, 64, 1)])
-def test_bisection_small_shapes(N, D, H):
+@pytest.mark.parametrize("N,D,H,leaf", [(128, 64, 1, 64), (512, 128, 2, 64), (4096, 64, 1, 64), (2048, 128, 2, 32),
+                                         (1024, 64, 1, 128)])
+def test_bisection_small_shapes(N, D, H, leaf):
     w = synth.WORKLOADS["unstructured"].with_(N=N, D=D, H=H, d_split=(D, 0, 0), components=16, k_min=32,
-                                               config_id=150 + N, c_q=N // 64, c_sub=(N // 64, 1, 1))
+                                               config_id=150 + N, c_q=N // leaf, c_sub=(N // leaf, 1, 1),
+                                               fixed_cluster_size=leaf)
     bisect_parity(w, range(H))
 
 
