@@ -66,7 +66,6 @@ struct Args {
     const int32_t *indices;
     const int32_t *n_c;        // [BH][Cq] or null
     int32_t *err;
-    float *lse;                // [BH][N] natural log-sum-exp of every stored row, or null
     // Grouped work items (ClusterAttention leaves of 32 or 64 queries): item =
     // (bh, group of L consecutive leaves), `indices` holds the groups' union
     // lists at their first leaf's offset, u_n their lengths, and gmask the
@@ -74,11 +73,25 @@ struct Args {
     const uint32_t *gmask;
     const int32_t *u_n;
     int L, leaf_shift, G;
+    // Compensation of excluded key clusters (ClusterAttention, compensate = 1):
+    // after its listed keys a work item walks "virtual" keys, one per key
+    // cluster k with members outside a leaf's list, whose key and value are
+    // the cluster's mean key mu_k and mean value vbar_k (each as a bf16
+    // hi + lo pair, summed by two MMAs) and whose logit carries log2(m_k),
+    // m_k the leaf's excluded members of k (-inf where m_k = 0).  Virtual
+    // tiles hold 64 keys: rows 0-63 of a K/V stage the hi halves, 64-127 the
+    // lo halves.  Per virtual group vg (the work item's group, or its cluster
+    // when ungrouped): vn[vg] keys in tiles vg*vtiles .. of vlist (key
+    // cluster ids, 64 per tile) and vbias ([tile][leaf][64]).
+    const __nv_bfloat16 *vk_hi, *vk_lo, *vv_hi, *vv_lo;  // [BH][Ck][D]
+    const int32_t *vlist, *vn;
+    const float *vbias;
+    int Ck, Lv, vtiles;
     int N, Cq;
     float scale_log2;          // log2(e) / sqrt(D)
 };
 
-template <int D, bool GROUPED>
+template <int D, bool GROUPED, bool COMP>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(Args a)
 {
@@ -124,6 +137,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long mslot = GROUPED ? loff / 128 + item : 0;
     if (GROUPED && nk <= 0) return;  // uniform; a group's leaves always hold keys
     const int ntiles = (nk + BN - 1) / BN;
+    // virtual tiles (compensation) follow the listed keys' tiles
+    const int64_t vg = GROUPED ? (int64_t)item : (int64_t)bh * a.Cq + c;
+    const int64_t vt0 = COMP ? vg * a.vtiles : 0;
+    const int ttot = ntiles + (COMP ? (a.vn[vg] + 63) / 64 : 0);
 
     if (threadIdx.x == 0) {
         // producer and softmax barriers take one arrival per warp (lane 0,
@@ -176,6 +193,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int NR = BN / RPI;
         int keys[NR];
         auto load_keys = [&](int j) {
+            if (COMP && j >= ntiles) {
+                // virtual tile: rows r and r + 64 take slot r & 63 (padding
+                // slots repeat a real cluster and carry a -inf bias)
+#pragma unroll
+                for (int i = 0; i < NR; ++i) keys[i] = a.vlist[(vt0 + j - ntiles) * 64 + ((i * RPI + r0) & 63)];
+                return;
+            }
 #pragma unroll
             for (int i = 0; i < NR; ++i) {
                 const int kj = min(j * BN + i * RPI + r0, nk - 1);
@@ -189,12 +213,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cp_async16(dst + sw_off(i * RPI + r0, ch, BN), src + keys[i] * sn + ch * 8, true);
             cp_async_commit();
         };
+        // virtual tiles: rows 0-63 the bf16 hi halves, rows 64-127 the lo halves
+        auto issue_virtual = [&](unsigned char *dst_base, const __nv_bfloat16 *hi, const __nv_bfloat16 *lo, int j) {
+            const uint32_t dst = smem_u32(dst_base + (j & 1) * KV_BYTES);
+            const int64_t tb = (int64_t)bh * a.Ck * D;
+#pragma unroll
+            for (int i = 0; i < NR; ++i)
+                cp_async16(dst + sw_off(i * RPI + r0, ch, BN), (i * RPI < 64 ? hi : lo) + tb + (int64_t)keys[i] * D + ch * 8,
+                           true);
+            cp_async_commit();
+        };
         const __nv_bfloat16 *kbh = a.kr + base * D;
+        auto issue_k = [&](int j) {
+            if (COMP && j >= ntiles) issue_virtual(sK, a.vk_hi, a.vk_lo, j);
+            else issue(sK, kbh, D, j);
+        };
+        auto issue_v = [&](int j) {
+            if (COMP && j >= ntiles) issue_virtual(sV, a.vv_hi, a.vv_lo, j);
+            else issue(sV, vbh, vsn, j);
+        };
         load_keys(0);
-        issue(sK, kbh, D, 0);
-        issue(sV, vbh, vsn, 0);
-        for (int j = 0; j < ntiles; ++j) {
-            const bool more = j + 1 < ntiles;
+        issue_k(0);
+        issue_v(0);
+        for (int j = 0; j < ttot; ++j) {
+            const bool more = j + 1 < ttot;
             // in flight: K(j), V(j)
             cp_async_wait1();
             fence_async_smem();
@@ -205,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j + 1 >= 2 && !mbar_wait(&bar_k_empty[(j + 1) & 1], (((j + 1) >> 1) - 1) & 1, abort_flag, a.err,
                                              0x10))
                     break;
-                issue(sK, kbh, D, j + 1);
+                issue_k(j + 1);
                 cp_async_wait1();  // in flight: V(j), K(j+1)
             } else {
                 cp_async_wait_all();
@@ -217,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j + 1 >= 2 && !mbar_wait(&bar_v_empty[(j + 1) & 1], (((j + 1) >> 1) - 1) & 1, abort_flag, a.err,
                                              0x11))
                     break;
-                issue(sV, vbh, vsn, j + 1);
+                issue_v(j + 1);
             }
         }
         cp_async_wait_all();
@@ -225,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16(BN, false);
+            const uint32_t id_qk64 = idesc_bf16(64, false);
             const uint32_t id_pv = idesc_bf16(D, true);
             const int nt = two ? 2 : 1;
             // descriptors of the first tile / stage; the start-address field
@@ -235,10 +278,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto issue_qk = [&](int t, int j) {
                 const uint64_t aq = dq + (uint64_t)((t * QT_BYTES) >> 4);
                 const uint64_t bk = dk + (uint64_t)(((j & 1) * KV_BYTES) >> 4);
+                if (COMP && j >= ntiles) {
+                    // S[:, 0:64] = Q (K_hi + K_lo)^T: N = 64 over rows 0-63, then rows 64-127
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k)
-                    mma_ss(tmem + t * 128, aq + (uint64_t)(((k >> 2) * (BM * 128) + (k & 3) * 32) >> 4),
-                           bk + (uint64_t)(((k >> 2) * (BN * 128) + (k & 3) * 32) >> 4), id_qk, k > 0);
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k)
+                            mma_ss(tmem + t * 128, aq + (uint64_t)(((k >> 2) * (BM * 128) + (k & 3) * 32) >> 4),
+                                   bk + (uint64_t)(((k >> 2) * (BN * 128) + h * 64 * 128 + (k & 3) * 32) >> 4),
+                                   id_qk64, h > 0 || k > 0);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_ss(tmem + t * 128, aq + (uint64_t)(((k >> 2) * (BM * 128) + (k & 3) * 32) >> 4),
+                               bk + (uint64_t)(((k >> 2) * (BN * 128) + (k & 3) * 32) >> 4), id_qk, k > 0);
+                }
                 mma_commit(&bar_s_full[t]);
                 if (t == nt - 1) mma_commit(&bar_k_empty[j & 1]);
             };
@@ -248,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 for (int t = 0; t < nt; ++t) issue_qk(t, 0);
             }
-            for (int j = 0; ok && j < ntiles; ++j) {
+            for (int j = 0; ok && j < ttot; ++j) {
                 const int s = j & 1;
                 if (!mbar_wait(&bar_v_full[s], (j >> 1) & 1, abort_flag, a.err, 0x24)) break;
                 const uint64_t bv = dv + (uint64_t)((s * KV_BYTES) >> 4);
@@ -258,12 +312,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
+                    if (COMP && j >= ntiles) {
+                        // O += P[:, 0:64] (V_hi + V_lo): P's first 64 keys against rows 0-63, then 64-127
 #pragma unroll
-                    for (int k = 0; k < BN / 16; ++k)
-                        mma_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, bv + (uint64_t)((k * 2048) >> 4), id_pv,
-                               (j > 0 || k > 0));
+                        for (int k = 0; k < 8; ++k)
+                            mma_ts(tmem + 256 + t * 128, tmem + t * 128 + (k & 3) * 8, bv + (uint64_t)((k * 2048) >> 4),
+                                   id_pv, true);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < BN / 16; ++k)
+                            mma_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, bv + (uint64_t)((k * 2048) >> 4),
+                                   id_pv, (j > 0 || k > 0));
+                    }
                     if (t == nt - 1) mma_commit(&bar_v_empty[s]);
-                    if (j + 1 < ntiles) {
+                    if (j + 1 < ttot) {
                         if (t == 0 && !mbar_wait(&bar_k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.err,
                                                  0x23)) {
                             ok = false;
@@ -292,23 +354,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint4 *gm = GROUPED ? reinterpret_cast<const uint4 *>(a.gmask) + mslot * a.L +
                                         ((t * BM + row) >> a.leaf_shift)
                                   : nullptr;
-        for (int j = 0; ok && j < ntiles; ++j) {
-            uint4 mw;
-            if constexpr (GROUPED) mw = __ldg(gm + (int64_t)j * a.L);  // in flight during the wait
+        // compensation: this row's leaf among the virtual group's bias rows
+        const int leaf_v = GROUPED ? ((t * BM + row) >> a.leaf_shift) : 0;
+        for (int j = 0; ok && j < ttot; ++j) {
+            const bool virt = COMP && j >= ntiles;
+            uint4 mw = make_uint4(~0u, ~0u, ~0u, ~0u);
+            if (GROUPED && !virt) mw = __ldg(gm + (int64_t)j * a.L);  // in flight during the wait
             if (!mbar_wait(&bar_s_full[t], j & 1, abort_flag, a.err, 0x30 + t)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const int valid = min(BN, nk - j * BN);
             uint32_t r[BN];
 #pragma unroll
             for (int c4 = 0; c4 < BN / 32; ++c4) tmem_ld32(tS + c4 * 32, r + c4 * 32);
             tmem_wait_ld();
-            if (valid < BN) {
+            if (virt) {
+                // 64 virtual keys: the raw logit plus ln(m) * sqrt(D) (so that
+                // the scaled exponent gains log2 m), -inf for m = 0, padding
+                // slots and the unused columns 64-127
+                const float4 *bq =
+                    reinterpret_cast<const float4 *>(a.vbias + ((vt0 + j - ntiles) * a.Lv + leaf_v) * 64);
 #pragma unroll
-                for (int i = 0; i < BN; ++i)
-                    if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const float4 b = __ldg(bq + c4);
+                    r[4 * c4 + 0] = __float_as_uint(__uint_as_float(r[4 * c4 + 0]) + b.x);
+                    r[4 * c4 + 1] = __float_as_uint(__uint_as_float(r[4 * c4 + 1]) + b.y);
+                    r[4 * c4 + 2] = __float_as_uint(__uint_as_float(r[4 * c4 + 2]) + b.z);
+                    r[4 * c4 + 3] = __float_as_uint(__uint_as_float(r[4 * c4 + 3]) + b.w);
+                }
+#pragma unroll
+                for (int i = 64; i < BN; ++i) r[i] = __float_as_uint(-INFINITY);
+            } else {
+                const int valid = min(BN, nk - j * BN);
+                if (valid < BN) {
+#pragma unroll
+                    for (int i = 0; i < BN; ++i)
+                        if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+                }
             }
             if constexpr (GROUPED) {
                 if ((mw.x & mw.y & mw.z & mw.w) != ~0u) {  // warp-uniform: a warp's rows share a leaf
@@ -393,8 +476,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool store = qi < nq;
             const int tok = store ? (a.perm ? a.perm[base + cstart + q0 + qi] : q0 + qi) : 0;
             const float inv = 1.f / l;
-            // row log-sum-exp, natural log: the row's exponentials are 2^(s*scale*log2e - m_run)
-            if (a.lse && store) a.lse[base + tok] = (m_run + log2f(l)) * 0.6931471805599453f;
             __nv_bfloat16 *dst = a.o + a.os.row(bh, tok);
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
@@ -459,20 +540,32 @@ constexpr size_t tc_smem_bytes(int D)
     return need > 120 * 1024 ? need : 120 * 1024;
 }
 
+template <int D, bool G, bool C>
+static cudaError_t attn_attr()
+{
+    return cudaFuncSetAttribute(tc::attn_tc_kernel<D, G, C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)tc_smem_bytes(D));
+}
+
 cudaError_t attn_tc_configure()
 {
-    cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tc_smem_bytes(128));
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc::attn_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tc_smem_bytes(64));
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc::attn_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tc_smem_bytes(128));
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc::attn_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tc_smem_bytes(64));
-    return e;
+    const cudaError_t e[8] = {attn_attr<128, false, false>(), attn_attr<64, false, false>(),
+                              attn_attr<128, true, false>(),  attn_attr<64, true, false>(),
+                              attn_attr<128, false, true>(),  attn_attr<64, false, true>(),
+                              attn_attr<128, true, true>(),   attn_attr<64, true, true>()};
+    for (cudaError_t x : e)
+        if (x != cudaSuccess) return x;
+    return cudaSuccess;
+}
+
+template <int D>
+static void attn_launch(const tc::Args &a, bool grouped, bool comp, int grid, cudaStream_t st)
+{
+    const size_t sm = tc_smem_bytes(D);
+    if (grouped && comp) tc::attn_tc_kernel<D, true, true><<<grid, tc::kThreads, sm, st>>>(a);
+    else if (grouped) tc::attn_tc_kernel<D, true, false><<<grid, tc::kThreads, sm, st>>>(a);
+    else if (comp) tc::attn_tc_kernel<D, false, true><<<grid, tc::kThreads, sm, st>>>(a);
+    else tc::attn_tc_kernel<D, false, false><<<grid, tc::kThreads, sm, st>>>(a);
 }
 
 int attn_tc_max_items(int BH, int N, int Cq) { return BH * ((N + 2 * tc::BM - 1) / (2 * tc::BM) + Cq); }
@@ -503,8 +596,8 @@ bool rows_tensor_map(CUtensorMap *m, const void *base, uint64_t rows, int D, int
 bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv_bfloat16 *v, const RowStrides &vs,
                     __nv_bfloat16 *o, const RowStrides &os, int4 *items, int32_t *n_items, int max_items, const int32_t *sizes, const int32_t *perm,
                     const int32_t *start, const long long *offsets, const int32_t *indices, const int32_t *n_c,
-                    int32_t *err, float *lse, int BH, int N, int D, int Cq, cudaStream_t st,
-                    const GroupedLists *grouped)
+                    int32_t *err, int BH, int N, int D, int Cq, cudaStream_t st,
+                    const GroupedLists *grouped, const CompLists *comp)
 {
     if (grouped) {
         max_items = BH * (Cq / grouped->L);
@@ -512,7 +605,7 @@ bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv
         tc::tc_items_kernel<<<1, 1024, 0, st>>>(sizes, items, n_items, BH, sizes ? Cq : 1, N);
         count_launches(1);
     }
-    tc::Args a;
+    tc::Args a{};
     a.qr = qr;
     a.kr = kr;
     a.v = v;
@@ -527,24 +620,29 @@ bool launch_attn_tc(const __nv_bfloat16 *qr, const __nv_bfloat16 *kr, const __nv
     a.indices = indices;
     a.n_c = n_c;
     a.err = err;
-    a.lse = lse;
     a.gmask = grouped ? grouped->masks : nullptr;
     a.u_n = grouped ? grouped->u_n : nullptr;
     a.L = grouped ? grouped->L : 0;
     a.leaf_shift = grouped ? grouped->leaf_shift : 0;
     a.G = grouped ? Cq / grouped->L : 0;
     if (grouped) a.indices = grouped->u_idx;
+    if (comp) {
+        a.vk_hi = comp->vk_hi;
+        a.vk_lo = comp->vk_lo;
+        a.vv_hi = comp->vv_hi;
+        a.vv_lo = comp->vv_lo;
+        a.vlist = comp->vlist;
+        a.vn = comp->vn;
+        a.vbias = comp->vbias;
+        a.Ck = comp->Ck;
+        a.Lv = comp->Lv;
+        a.vtiles = comp->vtiles;
+    }
     a.N = N;
     a.Cq = Cq;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-    if (D == 128 && grouped)
-        tc::attn_tc_kernel<128, true><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(a);
-    else if (D == 128)
-        tc::attn_tc_kernel<128, false><<<max_items, tc::kThreads, tc_smem_bytes(128), st>>>(a);
-    else if (grouped)
-        tc::attn_tc_kernel<64, true><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(a);
-    else
-        tc::attn_tc_kernel<64, false><<<max_items, tc::kThreads, tc_smem_bytes(64), st>>>(a);
+    if (D == 128) attn_launch<128>(a, grouped != nullptr, comp != nullptr, max_items, st);
+    else attn_launch<64>(a, grouped != nullptr, comp != nullptr, max_items, st);
     count_launches(1);
     return true;
 }

@@ -47,6 +47,17 @@ struct GroupedLists {
     int L, leaf_shift;
 };
 
+// Virtual keys of the ClusterAttention compensation (virt.cu): per virtual
+// group (a grouped work item, else a query cluster) up to vtiles tiles of 64
+// excluded key clusters, with per-leaf logit biases.
+struct CompLists {
+    const __nv_bfloat16 *vk_hi, *vk_lo, *vv_hi, *vv_lo;  // [BH][Ck][D] mean key / value, bf16 hi + lo
+    const int32_t *vlist;  // [groups][vtiles * 64] key clusters
+    const int32_t *vn;     // [groups] virtual keys per group
+    const float *vbias;    // [groups][vtiles][Lv][64] ln(m) * sqrt(D), or -inf
+    int Ck, Lv, vtiles;
+};
+
 struct RowStrides {
     int64_t sB, sH, sN;
     int H;

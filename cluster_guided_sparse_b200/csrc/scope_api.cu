@@ -43,15 +43,17 @@ cudaError_t attn_tc_configure();
 int attn_tc_max_items(int BH, int N, int Cq);
 bool launch_attn_tc(const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, const RowStrides &,
                     __nv_bfloat16 *, const RowStrides &, int4 *, int32_t *, int, const int32_t *, const int32_t *,
-                    const int32_t *, const long long *, const int32_t *, const int32_t *, int32_t *, float *, int, int,
-                    int, int, cudaStream_t, const GroupedLists *);
+                    const int32_t *, const long long *, const int32_t *, const int32_t *, int32_t *, int, int, int, int,
+                    cudaStream_t, const GroupedLists *, const CompLists *);
 size_t pack_mask_bytes(int64_t cap, int BH, int G, int L);
 void launch_pack_lists(const long long *, const int32_t *, const int32_t *, int32_t *, int32_t *, uint32_t *, int, int,
                        int, int, cudaStream_t);
-void launch_compensate(const __nv_bfloat16 *, const __nv_bfloat16 *, const RowStrides &, const int32_t *,
-                       const int32_t *, const int32_t *, const int32_t *, const int32_t *, const int32_t *,
-                       const float *, float *, const long long *, const int32_t *, const int32_t *, const float *,
-                       __nv_bfloat16 *, const RowStrides &, int, int, int, int, int, cudaStream_t);
+int virt_tiles(int Ck);
+void launch_virt_plan(const float *, __nv_bfloat16 *, __nv_bfloat16 *, const long long *, const int32_t *,
+                      const int32_t *, const int32_t *, const int32_t *, int32_t *, int32_t *, float *, int, int, int, int,
+                      int, int, cudaStream_t);
+void launch_vmean(const __nv_bfloat16 *, const RowStrides &, const int32_t *, const int32_t *, __nv_bfloat16 *,
+                  __nv_bfloat16 *, int, int, int, int, cudaStream_t);
 void launch_wait_timeout(int32_t *err, long long limit, cudaStream_t st);
 void run_selection(const float *lut, const int32_t *codes, const int32_t *item_id, const int32_t *item_cnt,
                    const int32_t *item_n, const uint16_t *key_item, int Pcap, int N, int Cq, int Ct, int Ch, int Cw,
@@ -102,7 +104,9 @@ struct Layout {
     size_t qr, kr, qnorm, ksub2, kchi, kclo, kfix, tab, stats, maxabs, q_lab, q_cent, q_cn, q_sizes, q_perm, q_start, q_bhist, q_tsum;
     size_t k_codes, k_cent[3], k_cn[3], k_sizes[3], k_perm[3], k_start[3], k_bhist[3], k_tsum[3];
     size_t sel_state, eg_state, lut, item_hist, item_id, item_cnt, item_n, key_item, r, n, kh, offsets, indices, work, nwork, vb, fix;
-    size_t bis_order, bis_delta, bis_aux, q_chi, q_clo, q_sums, k_sums[3], sums_bytes, lse, vmean;
+    size_t bis_order, bis_delta, bis_aux, q_chi, q_clo, q_sums, k_sums[3], sums_bytes;
+    size_t vk_hi, vk_lo, vv_hi, vv_lo, vlist, vn, vbias;  // compensation's virtual keys (comp)
+    int Lv, vtiles;                                        // leaves per virtual group, tiles per group
     size_t u_idx, u_n, gmask;  // grouped attention lists (gL > 0)
     int gL, gshift, G;         // leaves per group, log2(leaf), groups per head
     bool comp, eg, blocks;
@@ -369,8 +373,6 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.bis_delta = take(cur, L.bisect ? BH * N * 8 : 0);
     L.bis_aux = take(cur, L.bisect ? bisect_aux_bytes((int)BH, (int)N, (int)D) : 0);
     L.comp = p->compensate != 0;
-    L.lse = take(cur, L.comp ? BH * N * 4 : 0);
-    L.vmean = take(cur, L.comp ? BH * L.C[0] * D * 4 : 0);
     L.k_codes = take(cur, 3 * BH * N * 4);
     for (int s = 0; s < 3; ++s) {
         L.k_cent[s] = take(cur, BH * L.C[s] * (L.ds[s] > 0 ? L.ds[s] : 1) * 4);
@@ -412,6 +414,21 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.u_idx = take(cur, L.gL ? (size_t)L.cap * 4 : 0);
     L.u_n = take(cur, L.gL ? (size_t)BH * L.G * 4 : 0);
     L.gmask = take(cur, L.gL ? pack_mask_bytes(L.cap, (int)BH, L.G, L.gL) : 0);
+    // compensation: virtual groups follow the attention's work items (a
+    // group of leaves when grouped, else one query cluster)
+    L.Lv = L.gL ? L.gL : 1;
+    L.vtiles = L.comp ? virt_tiles(L.C[0]) : 0;
+    {
+        const size_t tabs = L.comp ? (size_t)BH * L.C[0] * D * 2 : 0;
+        const size_t groups = L.comp ? (size_t)BH * (L.Cq / L.Lv) : 0;
+        L.vk_hi = take(cur, tabs);
+        L.vk_lo = take(cur, tabs);
+        L.vv_hi = take(cur, tabs);
+        L.vv_lo = take(cur, tabs);
+        L.vlist = take(cur, groups * L.vtiles * 64 * 4);
+        L.vn = take(cur, groups * 4);
+        L.vbias = take(cur, groups * L.vtiles * L.Lv * 64 * 4);
+    }
     L.total = cur;
     return L;
 }
@@ -658,6 +675,12 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
         launch_pack_lists(at<long long>(ws, L.offsets), at<int32_t>(ws, L.n), at<int32_t>(ws, L.indices),
                           at<int32_t>(ws, L.u_idx), at<int32_t>(ws, L.u_n), at<uint32_t>(ws, L.gmask), (int)BH, L.Cq,
                           L.gL, (int)N, s);
+    if (L.comp)
+        launch_virt_plan(at<float>(ws, L.k_cent[0]), at<__nv_bfloat16>(ws, L.vk_hi), at<__nv_bfloat16>(ws, L.vk_lo),
+                         at<long long>(ws, L.offsets), at<int32_t>(ws, L.n), at<int32_t>(ws, L.indices),
+                         at<int32_t>(ws, L.k_codes), at<int32_t>(ws, L.k_sizes[0]), at<int32_t>(ws, L.vlist),
+                         at<int32_t>(ws, L.vn), at<float>(ws, L.vbias), (int)BH, (int)N, (int)D, L.Cq, L.C[0], L.Lv,
+                         s);
     if ((st = launch_status("selection")) != SCOPE_OK) return st;
 
     scope_plan_s *h = (scope_plan_s *)malloc(sizeof(scope_plan_s));
@@ -718,21 +741,20 @@ extern "C" scope_status scope_attn(const scope_tensor *q, const scope_tensor *k,
     const RowStrides os = rows_of(o);
     const GroupedLists grouped{at<int32_t>(ws, L.u_idx), at<int32_t>(ws, L.u_n), at<uint32_t>(ws, L.gmask), L.gL,
                                L.gshift};
+    const CompLists comp{at<__nv_bfloat16>(ws, L.vk_hi), at<__nv_bfloat16>(ws, L.vk_lo),
+                         at<__nv_bfloat16>(ws, L.vv_hi), at<__nv_bfloat16>(ws, L.vv_lo),
+                         at<int32_t>(ws, L.vlist), at<int32_t>(ws, L.vn), at<float>(ws, L.vbias),
+                         L.C[0], L.Lv, L.vtiles};
+    if (L.comp)  // mean values of the key clusters: the compensation's virtual values
+        launch_vmean(vb, vs, at<int32_t>(ws, L.k_perm[0]), at<int32_t>(ws, L.k_start[0]),
+                     at<__nv_bfloat16>(ws, L.vv_hi), at<__nv_bfloat16>(ws, L.vv_lo), (int)L.BH, (int)L.N, (int)L.D,
+                     L.C[0], s);
     if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, vs, (__nv_bfloat16 *)o->ptr, os,
                    at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, at<int32_t>(ws, L.q_sizes),
                    at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start), at<long long>(ws, L.offsets),
                    at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n), at<int32_t>(ws, L.stats) + 4,
-                   L.comp ? at<float>(ws, L.lse) : nullptr, (int)L.BH, (int)L.N, (int)L.D, L.Cq, s,
-                   L.gL ? &grouped : nullptr))
+                   (int)L.BH, (int)L.N, (int)L.D, L.Cq, s, L.gL ? &grouped : nullptr, L.comp ? &comp : nullptr))
         return fail(SCOPE_ECUDA, "scope_attn: tensor map encoding failed");
-    if (L.comp)
-        // ClusterAttention: excluded key clusters enter through their mean key and value
-        launch_compensate(at<__nv_bfloat16>(ws, L.qr), vb, vs, at<int32_t>(ws, L.q_perm), at<int32_t>(ws, L.q_start),
-                          at<int32_t>(ws, L.k_perm[0]), at<int32_t>(ws, L.k_start[0]), at<int32_t>(ws, L.k_codes),
-                          at<int32_t>(ws, L.k_sizes[0]), at<float>(ws, L.k_cent[0]), at<float>(ws, L.vmean),
-                          at<long long>(ws, L.offsets), at<int32_t>(ws, L.indices), at<int32_t>(ws, L.n),
-                          at<float>(ws, L.lse), (__nv_bfloat16 *)o->ptr, os, (int)L.BH, (int)L.N, (int)L.D, L.Cq,
-                          L.C[0], s);
     return launch_status("scope_attn");
 }
 
@@ -809,8 +831,8 @@ extern "C" scope_status scope_dense_attn(const scope_tensor *q, const scope_tens
     const __nv_bfloat16 *vb = v_bf16(L, ws, v, &vs, s);
     if (!launch_attn_tc(at<__nv_bfloat16>(ws, L.qr), at<__nv_bfloat16>(ws, L.kr), vb, vs, (__nv_bfloat16 *)o->ptr,
                         rows_of(o), at<int4>(ws, L.work), at<int32_t>(ws, L.nwork), L.max_work, nullptr, nullptr, nullptr,
-                        nullptr, nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, nullptr, (int)L.BH, (int)L.N,
-                        (int)L.D, 1, s, nullptr))
+                        nullptr, nullptr, nullptr, at<int32_t>(ws, L.stats) + 4, (int)L.BH, (int)L.N,
+                        (int)L.D, 1, s, nullptr, nullptr))
         return fail(SCOPE_ECUDA, "scope_dense_attn: tensor map encoding failed");
     return launch_status("scope_dense_attn");
 }

@@ -108,7 +108,9 @@ typedef struct {
  *                  m_ck members of key cluster k missing from query cluster
  *                  c's list add m_ck * e^{q.mu_k/sqrt(D)} to the softmax
  *                  denominator and that times the mean value to the
- *                  numerator.
+ *                  numerator.  The attention computes these terms in the
+ *                  same online softmax, as extra keys (mu_k, vbar_k) whose
+ *                  logits carry ln m_ck.
  *   eg_tau, eg_group  EG-Sparse routing ("EG-Sparse", abstract: low-entropy
  *                  heads go to a grouped cross-head pool, high-entropy heads
  *                  keep per-row selection).  eg_tau <= 0: off (plain SCOPE
