@@ -269,7 +269,9 @@ struct KkArgs {
     int N, off1, off2, ncols;     // column offsets of the h and w centroids; used columns
 };
 
-template <int D>
+// A8: the subspace boundaries and the used columns are multiples of 8, so
+// only every eighth column can close a subspace or end the row.
+template <int D, bool A8>
 __global__ void __launch_bounds__(kKT, kMinBlocks)
     km_assign_keys_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmHi,
                              const __grid_constant__ CUtensorMap tmLo, KkArgs a)
@@ -376,13 +378,16 @@ __global__ void __launch_bounds__(kKT, kMinBlocks)
             a1[0] = a1[1] = a1[2] = 0;
 #pragma unroll
             for (int j = 0; j < 128; ++j) {
-                if (j == a.off1) {
-                    b1[0] = B1; b2[0] = B2; a1[0] = A1;
-                    B1 = B2 = INF;
-                }
-                if (j == a.off2) {
-                    b1[1] = B1; b2[1] = B2; a1[1] = A1;
-                    B1 = B2 = INF;
+                if (A8 && (j & 7) == 0 && j >= a.ncols) break;  // padding columns: +inf
+                if (!A8 || (j & 7) == 0) {
+                    if (j == a.off1) {
+                        b1[0] = B1; b2[0] = B2; a1[0] = A1;
+                        B1 = B2 = INF;
+                    }
+                    if (j == a.off2) {
+                        b1[1] = B1; b2[1] = B2; a1[1] = A1;
+                        B1 = B2 = INF;
+                    }
                 }
                 const float e = fmaf(-2.f, __uint_as_float(r[j]), cn_sh[j]);
                 B2 = fminf(B2, fmaxf(B1, e));  // an equal score keeps the lower index and a zero margin
@@ -448,10 +453,16 @@ cudaError_t km_tc_configure()
     cudaError_t e = cudaFuncSetAttribute(km_assign_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)((kMT + 2) * 128 * 128 * 2 + 1024));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(km_assign_keys_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(km_assign_keys_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (kMT + 2) * 128 * 128 * 2 + 1024);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(km_assign_keys_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (kMT + 2) * 128 * 64 * 2 + 1024);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(km_assign_keys_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)((kMT + 2) * 128 * 128 * 2 + 1024));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(km_assign_keys_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(km_assign_keys_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)((kMT + 2) * 128 * 64 * 2 + 1024));
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(km_assign_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -521,10 +532,12 @@ bool launch_km_assign_keys_tc(const KmProblem *P, __nv_bfloat16 *chi, __nv_bfloa
         return false;
     for (int s = 0; s < 3; ++s) cudaMemsetAsync(a.fix_count[s], 0, sizeof(int32_t), st);
     const dim3 grid((N + 128 * kMT - 1) / (128 * kMT), BH);
-    if (D == 128)
-        km_assign_keys_tc_kernel<128><<<grid, kKT, (kMT + 2) * 128 * 128 * 2 + 1024, st>>>(tmX, tmHi, tmLo, a);
-    else
-        km_assign_keys_tc_kernel<64><<<grid, kKT, (kMT + 2) * 128 * 64 * 2 + 1024, st>>>(tmX, tmHi, tmLo, a);
+    const bool a8 = a.off1 % 8 == 0 && a.off2 % 8 == 0 && a.ncols % 8 == 0;
+    const size_t sm = (size_t)(kMT + 2) * 128 * D * 2 + 1024;
+    if (D == 128 && a8) km_assign_keys_tc_kernel<128, true><<<grid, kKT, sm, st>>>(tmX, tmHi, tmLo, a);
+    else if (D == 128) km_assign_keys_tc_kernel<128, false><<<grid, kKT, sm, st>>>(tmX, tmHi, tmLo, a);
+    else if (a8) km_assign_keys_tc_kernel<64, true><<<grid, kKT, sm, st>>>(tmX, tmHi, tmLo, a);
+    else km_assign_keys_tc_kernel<64, false><<<grid, kKT, sm, st>>>(tmX, tmHi, tmLo, a);
     count_launches(1);
     return true;
 }

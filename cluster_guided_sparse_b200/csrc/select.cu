@@ -903,6 +903,9 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         g += wgt[w];
         e += weq[w];
     }
+    // staging rows (256 keys per warp step) in the select's bucket array,
+    // which the count select above no longer needs
+    int *stage = reinterpret_cast<int *>(S.met) + warp * 256;
     for (int j0 = j_begin; j0 < j_end; j0 += 256) {
         const int j = j0 + 8 * lane;
         uint8_t k[8];
@@ -923,24 +926,28 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         }
         const unsigned tot = __shfl_sync(0xffffffffu, incl, 31);
         const unsigned ex = incl - packed;
+        // Output slot of a selected key = selected keys before it: keys above
+        // the cut, plus keys at it up to `need`.  The step's selected keys
+        // land in this warp's staging row in order, then go out as coalesced
+        // 128-byte stores.
+        const unsigned base = g + min(e, (unsigned)need);  // selected keys before this step
         unsigned gl = g + (ex & 0xffffu), el = e + (ex >> 16);
+        unsigned pos = gl + min(el, (unsigned)need) - base;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            if (k[t] == 2) {
-                const unsigned slot = gl + (el < (unsigned)need ? el : (unsigned)need);
-                if (slot < (unsigned)n) out[slot] = j + t;
-                else set_error(a.err, kErrRange, 0x300 + c);
-                ++gl;
-            } else if (k[t] == 1) {
-                if (el < (unsigned)need) {
-                    if (gl + el < (unsigned)n) out[gl + el] = j + t;
-                    else set_error(a.err, kErrRange, 0x300 + c);
-                }
-                ++el;
-            }
+            const bool sel = k[t] == 2 || (k[t] == 1 && el < (unsigned)need);
+            if (k[t] == 1) ++el;
+            if (sel) stage[pos++] = j + t;
         }
         g += tot & 0xffffu;
         e += tot >> 16;
+        const unsigned step_sel = g + min(e, (unsigned)need) - base;
+        __syncwarp();
+        for (unsigned i = lane; i < step_sel; i += 32) {
+            if (base + i < (unsigned)n) out[base + i] = stage[i];
+            else set_error(a.err, kErrRange, 0x300 + c);
+        }
+        __syncwarp();
     }
 }
 
@@ -951,6 +958,7 @@ static size_t sel_smem(int Csum) { return (size_t)((Csum + 3) & ~3) * sizeof(flo
 cudaError_t select_configure()
 {
     static_assert(kItemCache * 4 >= kMaxItems, "the 64 KB region must hold a class byte per item");
+    static_assert(kBuckets * 2 >= (kSelThreads / 32) * 256, "emit stages 256 keys per warp in SelShared::met");
     const int max_csum = kMaxBlocks + 2 > 3 * kMaxClusters ? kMaxBlocks + 2 : 3 * kMaxClusters;
     cudaError_t e = cudaFuncSetAttribute(emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sel_smem(max_csum));
