@@ -129,15 +129,45 @@ __device__ __forceinline__ void select_k(BisectShared &S, const double *delta, i
 // only, gathered in shared memory.  A bucket holding more than kCoarseCap
 // keys falls back to the radix select over all n.
 constexpr int kCoarse = 4096, kCoarseCap = 2048;
-struct CoarseShared {
-    int hist[kCoarse];
-    unsigned long long list[kCoarseCap];
+template <int NB, int CAP>
+struct CoarseT {
+    int hist[NB];
+    unsigned long long list[CAP];
     double red[2][32];
     double lo, scale;
     int nlist, bucket, below;
 };
+using CoarseShared = CoarseT<kCoarse, kCoarseCap>;  // top-level nodes (one CTA per node)
+using CoarseSmall = CoarseT<2048, 32>;             // nodes of up to 1024 rows
 
-__device__ void select_k_coarse(BisectShared &S, CoarseShared &C, const double *delta, int n, int k, Cut &c)
+// The exact cut among m <= 32 keys, by one warp: a lane's key is the cut when
+// fewer than k keys are below it and at least k are at or below it.
+__device__ void small_select(BisectShared &S, const unsigned long long *list, int m, int k, Cut &c)
+{
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const unsigned long long u = lane < m ? list[lane] : ~0ull;
+        int lt = 0, le = 0;
+        for (int i = 0; i < m; ++i) {
+            const unsigned long long v = __shfl_sync(0xffffffffu, u, i);
+            lt += v < u ? 1 : 0;
+            le += v <= u ? 1 : 0;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, lane < m && lt < k && k <= le);
+        if (lane == __ffs(hit) - 1) {
+            S.prefix = u;
+            S.need = k - lt;
+            S.eq = le - lt;
+        }
+    }
+    __syncthreads();
+    c.key = S.prefix;
+    c.need = S.need;
+    c.eq = S.eq;
+}
+
+template <int NB, int CAP>
+__device__ void select_k_coarse(BisectShared &S, CoarseT<NB, CAP> &C, const double *delta, int n, int k, Cut &c)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     double lo = INFINITY, hi = -INFINITY;
@@ -154,7 +184,7 @@ __device__ void select_k_coarse(BisectShared &S, CoarseShared &C, const double *
         C.red[0][warp] = lo;
         C.red[1][warp] = hi;
     }
-    for (int b = tid; b < kCoarse; b += blockDim.x) C.hist[b] = 0;
+    for (int b = tid; b < NB; b += blockDim.x) C.hist[b] = 0;
     __syncthreads();
     if (tid == 0) {
         double l = C.red[0][0], h = C.red[1][0];
@@ -163,12 +193,12 @@ __device__ void select_k_coarse(BisectShared &S, CoarseShared &C, const double *
             h = fmax(h, C.red[1][w]);
         }
         C.lo = l;
-        C.scale = h > l ? (double)kCoarse / (h - l) : 0.0;
+        C.scale = h > l ? (double)NB / (h - l) : 0.0;
         C.nlist = 0;
     }
     __syncthreads();
     const double l = C.lo, sc = C.scale;
-    auto bucket_of = [&](double d) { return min(kCoarse - 1, (int)((d - l) * sc)); };
+    auto bucket_of = [&](double d) { return min(NB - 1, (int)((d - l) * sc)); };
     for (int i0 = 0; i0 < n; i0 += blockDim.x) {
         const int i = i0 + tid;
         const int b = i < n ? bucket_of(delta[i]) : -1;
@@ -178,20 +208,21 @@ __device__ void select_k_coarse(BisectShared &S, CoarseShared &C, const double *
     __syncthreads();
     // the first bucket where the running count reaches k: thread t scans
     // buckets [t*per, (t+1)*per) from its exclusive prefix
-    const int per = kCoarse / blockDim.x;  // blockDim divides 4096
+    const int per = (NB + blockDim.x - 1) / blockDim.x;
+    const int b0 = min(NB, tid * per), b1 = min(NB, b0 + per);
     int loc = 0;
-    for (int e = 0; e < per; ++e) loc += C.hist[tid * per + e];
+    for (int b = b0; b < b1; ++b) loc += C.hist[b];
     int tot;
     const int before = block_excl_scan(loc, S.tmp, tot);
     if (before < k && before + loc >= k) {
-        int acc = before, b = tid * per;
+        int acc = before, b = b0;
         for (; acc + C.hist[b] < k; ++b) acc += C.hist[b];
         C.bucket = b;
         C.below = acc;
     }
     __syncthreads();
     const int bk = C.bucket, below = C.below, m = C.hist[bk];
-    if (m > kCoarseCap) {
+    if (m > CAP) {
         select_k(S, delta, n, k, c);
         return;
     }
@@ -200,7 +231,8 @@ __device__ void select_k_coarse(BisectShared &S, CoarseShared &C, const double *
         if (bucket_of(d) == bk) C.list[atomicAdd(&C.nlist, 1)] = dkey(d);
     }
     __syncthreads();
-    radix_select(S, [&](int i) { return C.list[i]; }, m, k - below, c);
+    if (m <= 32) small_select(S, C.list, m, k - below, c);
+    else radix_select(S, [&](int i) { return C.list[i]; }, m, k - below, c);
 }
 
 // delta = ||x - c0||^2 - ||x - c1||^2 in fp64, dims in order.  The row is
@@ -344,6 +376,7 @@ template <int D>
 __global__ void __launch_bounds__(kBT) bisect_level_kernel(BisectArgs a)
 {
     __shared__ BisectShared S;
+    __shared__ CoarseSmall C;
     const int node = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     const int n = a.N >> a.level, half = n >> 1;
     const int lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
@@ -363,7 +396,7 @@ __global__ void __launch_bounds__(kBT) bisect_level_kernel(BisectArgs a)
         // delta of every member
         for (int i = tid; i < n; i += blockDim.x) delta[i] = split_delta<D>(X + (int64_t)mem[i] * D, S.c[0], S.c[1]);
         __syncthreads();
-        select_k(S, delta, n, half, cut);
+        select_k_coarse(S, C, delta, n, half, cut);
         if (r == a.iters) break;
         // mark sides, reusing delta as the side flag for the sums (a thread
         // reads and then overwrites only its own member's entry)
@@ -544,10 +577,12 @@ size_t bisect_aux_bytes(int BH, int N, int D)
 }
 
 // Bisection of every (bh) row set of X into N/leaf leaves.  `aux` holds
-// bisect_aux_bytes(BH, N, D) bytes (256-byte aligned).
+// bisect_aux_bytes(BH, N, D) bytes (256-byte aligned).  The BH row sets are
+// nout consecutive parts of BH / nout (the queries and the keys of a call,
+// bisected together so that the top levels' few nodes fill more of the
+// GPU); part p's leaves go to out[p].
 void launch_bisect(const __nv_bfloat16 *X, int BH, int N, int D, int leaf, int iters, int32_t *order,
-                   int32_t *order_tmp, double *delta, void *aux, int32_t *labels, float *cent, float *cn,
-                   int32_t *start, int32_t *sizes, int32_t *perm, cudaStream_t st)
+                   int32_t *order_tmp, double *delta, void *aux, const BisectOut *out, int nout, cudaStream_t st)
 {
     const int64_t total = (int64_t)BH * N;
     iota_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(order, N, total);
@@ -596,9 +631,14 @@ void launch_bisect(const __nv_bfloat16 *X, int BH, int N, int D, int leaf, int i
         cur = nxt;
         nxt = t;
     }
-    bisect_leaves_kernel<<<dim3(N / leaf, BH), 256, 0, st>>>(X, cur, N, D, leaf, labels, cent, cn, start, sizes,
-                                                             perm);
-    count_launches(1);
+    const int per = BH / nout;
+    for (int q = 0; q < nout; ++q) {
+        const BisectOut &o = out[q];
+        bisect_leaves_kernel<<<dim3(N / leaf, per), 256, 0, st>>>(X + (int64_t)q * per * N * D,
+                                                                  cur + (int64_t)q * per * N, N, D, leaf, o.labels,
+                                                                  o.cent, o.cn, o.start, o.sizes, o.perm);
+        count_launches(1);
+    }
 }
 
 }  // namespace scope

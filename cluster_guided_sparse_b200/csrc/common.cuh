@@ -58,6 +58,14 @@ struct CompLists {
     int Ck, Lv, vtiles;
 };
 
+// Outputs of a bisection part (bisect.cu): labels, leaf centroids and norms,
+// leaf starts and sizes, the leaf-major permutation.
+struct BisectOut {
+    int32_t *labels;
+    float *cent, *cn;
+    int32_t *start, *sizes, *perm;
+};
+
 struct RowStrides {
     int64_t sB, sH, sN;
     int H;

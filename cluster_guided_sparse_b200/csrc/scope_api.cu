@@ -25,8 +25,8 @@ cudaError_t km_configure();
 void launch_km_init(const KmBatch &, int, int, int, uint32_t, cudaStream_t);
 void launch_km_assign_direct(const KmBatch &, int, int, int, cudaStream_t);
 void launch_km_sort(const KmBatch &, int, int, cudaStream_t);
-void launch_bisect(const __nv_bfloat16 *, int, int, int, int, int, int32_t *, int32_t *, double *, void *, int32_t *,
-                   float *, float *, int32_t *, int32_t *, int32_t *, cudaStream_t);
+void launch_bisect(const __nv_bfloat16 *, int, int, int, int, int, int32_t *, int32_t *, double *, void *,
+                   const BisectOut *, int, cudaStream_t);
 size_t bisect_aux_bytes(int BH, int N, int D);
 cudaError_t km_tc_configure();
 bool launch_km_assign_tc(const KmProblem &, __nv_bfloat16 *, __nv_bfloat16 *, int, int, int, const float *, int32_t *,
@@ -341,8 +341,10 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
     L.cap = L.BH * L.Cq * L.N;
     const int64_t BH = L.BH, N = L.N, D = L.D;
     size_t cur = 0;
-    L.qr = take(cur, BH * N * D * 2);
-    L.kr = take(cur, BH * N * D * 2);
+    // Qr then Kr with no gap (a whole bisection runs over both as 2*BH row
+    // sets); BH*N*D*2 is a multiple of 128 bytes, so Kr stays aligned
+    L.qr = take(cur, 2 * BH * N * D * 2);
+    L.kr = L.qr + BH * N * D * 2;
     L.qnorm = take(cur, BH * N * 4);
     L.ksub2 = take(cur, BH * N * 16);
     L.kchi = take(cur, BH * 128 * D * 2);
@@ -369,9 +371,9 @@ Layout make_layout(const scope_tensor *q, const scope_grid *g, const scope_param
         for (int i = 0; i < 3; ++i) L.k_sums[i] = take(cur, BH * L.C[i] * (L.ds[i] > 0 ? L.ds[i] : 1) * 8);
         L.sums_bytes = cur - s0;
     }
-    L.bis_order = take(cur, L.bisect ? 2 * BH * N * 4 : 0);
-    L.bis_delta = take(cur, L.bisect ? BH * N * 8 : 0);
-    L.bis_aux = take(cur, L.bisect ? bisect_aux_bytes((int)BH, (int)N, (int)D) : 0);
+    L.bis_order = take(cur, L.bisect ? 4 * BH * N * 4 : 0);  // order + scratch for 2*BH row sets
+    L.bis_delta = take(cur, L.bisect ? 2 * BH * N * 8 : 0);
+    L.bis_aux = take(cur, L.bisect ? bisect_aux_bytes((int)(2 * BH), (int)N, (int)D) : 0);
     L.comp = p->compensate != 0;
     L.k_codes = take(cur, 3 * BH * N * 4);
     for (int s = 0; s < 3; ++s) {
@@ -572,15 +574,15 @@ extern "C" scope_status scope_plan(const scope_tensor *q, const scope_tensor *k,
         // ClusterAttention variant: balanced bisection of queries and of keys
         // into N / fixed_cluster_size clusters (one subspace = the full head dim).
         const int leaf = p->fixed_cluster_size;
+        // Qr and Kr are adjacent in the workspace: one bisection over 2*BH row sets
         int32_t *ord = at<int32_t>(ws, L.bis_order);
-        launch_bisect(at<__nv_bfloat16>(ws, L.qr), BH, N, D, leaf, p->iters, ord, ord + (int64_t)BH * N,
-                      at<double>(ws, L.bis_delta), ws + L.bis_aux, at<int32_t>(ws, L.q_lab),
-                      at<float>(ws, L.q_cent), at<float>(ws, L.q_cn), at<int32_t>(ws, L.q_start),
-                      at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.q_perm), s);
-        launch_bisect(at<__nv_bfloat16>(ws, L.kr), BH, N, D, leaf, p->iters, ord, ord + (int64_t)BH * N,
-                      at<double>(ws, L.bis_delta), ws + L.bis_aux, at<int32_t>(ws, L.k_codes),
-                      at<float>(ws, L.k_cent[0]), at<float>(ws, L.k_cn[0]), at<int32_t>(ws, L.k_start[0]),
-                      at<int32_t>(ws, L.k_sizes[0]), at<int32_t>(ws, L.k_perm[0]), s);
+        const BisectOut outs[2] = {
+            {at<int32_t>(ws, L.q_lab), at<float>(ws, L.q_cent), at<float>(ws, L.q_cn), at<int32_t>(ws, L.q_start),
+             at<int32_t>(ws, L.q_sizes), at<int32_t>(ws, L.q_perm)},
+            {at<int32_t>(ws, L.k_codes), at<float>(ws, L.k_cent[0]), at<float>(ws, L.k_cn[0]),
+             at<int32_t>(ws, L.k_start[0]), at<int32_t>(ws, L.k_sizes[0]), at<int32_t>(ws, L.k_perm[0])}};
+        launch_bisect(at<__nv_bfloat16>(ws, L.qr), 2 * BH, N, D, leaf, p->iters, ord, ord + 2 * (int64_t)BH * N,
+                      at<double>(ws, L.bis_delta), ws + L.bis_aux, outs, 2, s);
         cudaMemsetAsync(at<int32_t>(ws, L.k_codes) + (int64_t)BH * N, 0, (size_t)2 * BH * N * 4, s);
     } else {
     // Key subspaces always, and the queries when they have few clusters, run
