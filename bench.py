@@ -490,6 +490,34 @@ def run_scope(args, world, rank, local):
     gather_ms = max_over_ranks(statistics.mean(e[2].elapsed_time(e[3]) for e in ev), world)
     call_median_ms = max_over_ranks(statistics.median(e[0].elapsed_time(e[3]) for e in ev), world)
 
+    # The same call replayed from a CUDA graph (captured once; every replay
+    # runs every kernel of the plan and the attention on the same buffers):
+    # what a caller that captures the call pays, without the host-side
+    # launch cost that bounds the small workloads.
+    graph_ms = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                gp = scope.plan(qd, kd, params, grid, workspace=ws)
+                scope.attn(qd, kd, vd, gp, out=o)
+        stream.wait_stream(side)
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        gp.sync_status()
+        graph_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps, world)
+        del g
+
     # rows the final tensor-core query assignment sent to the fp64 re-check
     fix_rows = int(pl.view("fixup")[0]) if w.c_q >= 128 and w.fixed_cluster_size == 0 and w.block_kind == 0 else 0
     fix_rows = int(sum_over_ranks(fix_rows, world))
@@ -638,6 +666,7 @@ def run_scope(args, world, rank, local):
                    "parallelism": "single GPU" if world == 1 else
                    f"heads round-robin over {world} GPUs" + (", O all-gathered" if gather else "")},
         "effective_tflops": eff, "plan_ms": plan_ms, "attn_ms": attn_ms, "gather_ms": gather_ms,
+        "graph_ms": graph_ms,
         "call_median_ms": call_median_ms,
         "density": density, "density_per_head": [round(x, 4) for x in dens_h],
         "fidelity_vs_own_dense": {"rel_l2_mean": statistics.mean(rel_h), "rel_l2_max": max(rel_h),
@@ -676,6 +705,7 @@ def main():
     ap.add_argument("--eg-group", type=int, default=4)
     ap.add_argument("--no-gather", action="store_true", help="N > 1: leave the output heads sharded")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing (graph_ms)")
     ap.add_argument("--e2e-chunks", type=int, default=4,
                     help="head chunks of the end-to-end call (copies of one chunk overlap compute of another)")
     args = ap.parse_args()
