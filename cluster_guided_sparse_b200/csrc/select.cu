@@ -51,14 +51,14 @@ __global__ void __launch_bounds__(kLutThreads)
     lut_kernel(const float *qcent, const float *kc_t, const float *kc_h, const float *kc_w, float *lut, int Cq, int D,
                int dt, int dh, int dw, int Ct, int Ch, int Cw)
 {
-    extern __shared__ float lsm[];
+    extern __shared__ double lsm_d[];
     constexpr int QPT = kLutQ / kLutGroups;  // query centroids per thread
     const int c0 = blockIdx.x * kLutQ, bh = blockIdx.y;
     const int nq = min(kLutQ, Cq - c0);
-    float *q = lsm;                  // [kLutQ][D]
-    float *kt = lsm + kLutQ * D;     // [kLutRows][stride]
+    double *q = lsm_d;                                      // [kLutQ][D], converted once
+    float *kt = reinterpret_cast<float *>(lsm_d + kLutQ * D);  // [kLutRows][stride]
     for (int i = threadIdx.x; i < kLutQ * D; i += kLutThreads)
-        q[i] = i / D < nq ? qcent[((int64_t)bh * Cq + c0) * D + i] : 0.f;
+        q[i] = i / D < nq ? (double)qcent[((int64_t)bh * Cq + c0) * D + i] : 0.0;
     const int Csum = Ct + Ch + Cw;
     const int row = threadIdx.x % kLutRows, grp = threadIdx.x / kLutRows;
     const float *segs[3] = {kc_t, kc_h, kc_w};
@@ -78,11 +78,11 @@ __global__ void __launch_bounds__(kLutThreads)
 #pragma unroll
                 for (int u = 0; u < QPT; ++u) acc[u] = 0.0;
                 const float *kr = kt + row * stride;
-                const float *qs = q + grp * QPT * D + offs[s];
+                const double *qs = q + grp * QPT * D + offs[s];
                 for (int k = 0; k < ds; ++k) {
                     const double kv = (double)kr[k];
 #pragma unroll
-                    for (int u = 0; u < QPT; ++u) acc[u] += (double)qs[u * D + k] * kv;
+                    for (int u = 0; u < QPT; ++u) acc[u] += qs[u * D + k] * kv;
                 }
 #pragma unroll
                 for (int u = 0; u < QPT; ++u) {
@@ -959,6 +959,10 @@ cudaError_t select_configure()
 {
     static_assert(kItemCache * 4 >= kMaxItems, "the 64 KB region must hold a class byte per item");
     static_assert(kBuckets * 2 >= (kSelThreads / 32) * 256, "emit stages 256 keys per warp in SelShared::met");
+    // the table kernel's staging at D = 128: fp64 query centroids + one padded key tile
+    cudaError_t el = cudaFuncSetAttribute(lut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)(kLutQ * 128 * sizeof(double) + kLutRows * 129 * sizeof(float)));
+    if (el != cudaSuccess) return el;
     const int max_csum = kMaxBlocks + 2 > 3 * kMaxClusters ? kMaxBlocks + 2 : 3 * kMaxClusters;
     cudaError_t e = cudaFuncSetAttribute(emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sel_smem(max_csum));
@@ -977,7 +981,7 @@ void launch_lut(const float *qcent, const float *kc_t, const float *kc_h, const 
                 int Cq, int D, int dt, int dh, int dw, int Ct, int Ch, int Cw, cudaStream_t st)
 {
     const int dmax = max(dt, max(dh, dw));
-    const size_t smem = ((size_t)kLutQ * D + (size_t)kLutRows * (dmax | 1)) * sizeof(float);
+    const size_t smem = (size_t)kLutQ * D * sizeof(double) + (size_t)kLutRows * (dmax | 1) * sizeof(float);
     lut_kernel<<<dim3((Cq + kLutQ - 1) / kLutQ, BH), kLutThreads, smem, st>>>(qcent, kc_t, kc_h, kc_w, lut, Cq, D, dt,
                                                                              dh, dw, Ct, Ch, Cw);
     count_launches(1);
