@@ -350,12 +350,15 @@ def test_bisection_tied_rows(groups):
 # ClusterAttention compensation: every excluded key enters through its key
 # cluster's mean key and value (the oracle's attention_rows_comp, reading R16),
 # fed the device's own rotated rows, key-cluster labels and lists.
-@pytest.mark.parametrize("N,D,H,p", [(4096, 64, 2, 0.9), (4096, 64, 1, 0.5), (512, 128, 1, 0.9),
-                                     (65536, 64, 1, 0.9)])  # the benchmarked shape: 1024 key leaves
-def test_compensation_parity(N, D, H, p):
+@pytest.mark.parametrize("N,D,H,p,leaf", [(4096, 64, 2, 0.9, 64), (4096, 64, 1, 0.5, 64), (512, 128, 1, 0.9, 64),
+                                          (65536, 64, 1, 0.9, 64),  # the benchmarked shape: 1024 key leaves
+                                          (2048, 128, 1, 0.7, 32),  # eight leaves per work item
+                                          (4096, 64, 1, 0.7, 128),  # one leaf per work item (ungrouped)
+                                          (8192, 64, 1, 0.7, 512)])  # two work items per leaf
+def test_compensation_parity(N, D, H, p, leaf):
     w = synth.WORKLOADS["unstructured"].with_(N=N, D=D, H=H, d_split=(D, 0, 0), components=16, k_min=32,
-                                               config_id=170 + N + D, c_q=N // 64, c_sub=(N // 64, 1, 1),
-                                               top_p=p, compensate=1)
+                                               config_id=170 + N + D, c_q=N // leaf, c_sub=(N // leaf, 1, 1),
+                                               top_p=p, compensate=1, fixed_cluster_size=leaf)
     q, k, v = synth.make_inputs(w)
     qd, kd, vd = to_dev(q, k, v)
     pl = plan_of(w, qd, kd)
