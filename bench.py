@@ -613,10 +613,10 @@ def run_scope(args, world, rank, local):
     # The chunk count is the caller's choice: chunks overlap copies with
     # compute, but every chunk is a whole plan (its launches and fixed steps),
     # which launch-bound workloads pay once per chunk.  One untimed call with
-    # each candidate (1 and --e2e-chunks) picks the faster; every rank takes
-    # the same number of calls.
+    # each candidate (1, --e2e-chunks and twice that) picks the fastest; every
+    # rank takes the same number of calls.
     cands = []
-    for nc in (1, args.e2e_chunks):
+    for nc in (1, args.e2e_chunks, 2 * args.e2e_chunks):
         ch = split(nc)
         if ch not in [c for c, _ in cands]:
             ws_c = torch.empty(max(scope.workspace_bytes(qd[:, h0:h1], params, grid) for h0, h1 in ch),
@@ -626,7 +626,7 @@ def run_scope(args, world, rank, local):
     for ch, ws_c in cands:
         e2e_call(ch, ws_c)
         trial.append(e2e_call(ch, ws_c))
-    for _ in range(2 - len(cands)):  # the same number of calls on every rank
+    for _ in range(3 - len(cands)):  # the same number of calls on every rank
         e2e_call(*cands[0])
         e2e_call(*cands[0])
     chunks, ws_e2e = cands[min(range(len(cands)), key=lambda i: trial[i])]
@@ -707,7 +707,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing (graph_ms)")
     ap.add_argument("--e2e-chunks", type=int, default=4,
-                    help="head chunks of the end-to-end call (copies of one chunk overlap compute of another)")
+                    help="head chunks of the end-to-end call (copies of one chunk overlap compute of another); "
+                         "the bench also tries 1 and twice this and keeps the fastest")
     args = ap.parse_args()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         sys.exit(relaunch(args.gpus))
