@@ -200,10 +200,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < NR; ++i) keys[i] = a.vlist[(vt0 + j - ntiles) * 64 + ((i * RPI + r0) & 63)];
                 return;
             }
+            // the lists are read once: streaming loads (evict first from L2),
+            // so they do not push the head's K/V rows out of L2
 #pragma unroll
             for (int i = 0; i < NR; ++i) {
                 const int kj = min(j * BN + i * RPI + r0, nk - 1);
-                keys[i] = a.indices ? a.indices[loff + kj] : kj;
+                keys[i] = a.indices ? __ldcs(a.indices + loff + kj) : kj;
             }
         };
         auto issue = [&](unsigned char *dst_base, const __nv_bfloat16 *src, int64_t sn, int j) {
