@@ -4,11 +4,15 @@ include/scope.h declares, and rejects bad arguments before any device work.
 The pointers used here are fake, 16-byte aligned addresses: every call below
 must fail in argument validation, which runs before any CUDA call."""
 import ctypes
+import os
+import re
 
 import pytest
 
 import cluster_guided_sparse_b200 as scope
 from cluster_guided_sparse_b200 import build, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 FAKE = 0x7F0000000000  # aligned, never dereferenced
 
@@ -137,16 +141,28 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
         scope.lib()
 
 
-def test_compensation_workspace_holds_row_lse_and_cluster_means(L):
-    # ClusterAttention shape: N = 4096, 64-token clusters -> 64 key clusters, D = 64
+def test_compensation_workspace_holds_cluster_means_and_virtual_lists(L):
+    # ClusterAttention shape: N = 4096, 64-token clusters -> 64 key clusters, D = 64; leaves
+    # of 64 queries are grouped four to a work item (16 groups per head)
     w = synth.WORKLOADS["unstructured"].with_(N=4096, D=64, H=2, d_split=(64, 0, 0), c_q=64, c_sub=(64, 1, 1))
     q = T(N=4096, D=64, H=2)
     sizes = []
     for comp in (0, 1):
         p, g = scope.make_params(w, compensate=comp)
         sizes.append(L.scope_plan_workspace_bytes(ctypes.byref(q), ctypes.byref(g), ctypes.byref(p)))
-    BH, N, C, D = 2, 4096, 64, 64
-    assert sizes[0] > 0 and sizes[1] >= sizes[0] + BH * N * 4 + BH * C * D * 4
+    BH, C, D, groups, leaves, tiles = 2, 64, 64, 2 * 16, 4, 1
+    tables = 4 * BH * C * D * 2                    # mean keys and values, bf16 hi + lo
+    lists = groups * tiles * 64 * 4                # virtual key clusters
+    bias = groups * tiles * leaves * 64 * 4        # per-leaf logit offsets
+    assert sizes[0] > 0 and sizes[1] >= sizes[0] + tables + lists + bias
+
+
+def test_view_names_match_the_header():
+    hdr = open(os.path.join(ROOT, "include", "scope.h")).read()
+    ids = dict((m.group(1).lower(), int(m.group(2))) for m in re.finditer(r"SCOPE_VIEW_(\w+)\s*=\s*(\d+)", hdr))
+    count = ids.pop("count")
+    assert len(scope.VIEWS) == count
+    assert {name: i for i, name in enumerate(scope.VIEWS)} == ids
 
 
 def S(strides, N=256, D=64, H=2, B=1, dtype=scope.SCOPE_BF16):
