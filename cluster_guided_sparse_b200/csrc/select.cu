@@ -838,56 +838,58 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
             return;
         }
     }
-    // without cached keys, class every item once: 2 above, 1 at, 0 below the cut
-    uint8_t *cls = region;
-    if (!cached) {
-        for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
-            const uint32_t u = K(i);
-            cls[i] = u > key ? 2 : (u == key ? 1 : 0);
-        }
+    // every item's class once: 2 above the cut, 1 at it, 0 below (a byte per
+    // item after the 64 KB region; without cached keys, in the region itself)
+    uint8_t *cls = cached ? region + (size_t)kItemCache * 4 : region;
+    __syncthreads();  // the refine above may still read the cached keys
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const uint32_t u = K(i);
+        cls[i] = u > key ? 2 : (u == key ? 1 : 0);
     }
     __syncthreads();
-    auto class_of = [&](int item) -> uint8_t {
-        if (cached) {
-            const uint32_t u = cache[item];
-            return u > key ? 2 : (u == key ? 1 : 0);
-        }
-        return cls[item];
-    };
     // Key walk without block-wide scans: warp w owns a contiguous chunk of the
     // keys (a multiple of 256).  Each lane takes eight adjacent keys per step
-    // (one 16-byte load of their item ranks), so a warp step covers 256 keys.
-    // Pass 1 counts the chunk's keys above and at the cut in per-lane
-    // registers; after one barrier every warp knows its chunk's output base,
-    // and pass 2 walks the chunk again, placing each lane's keys after an
-    // exclusive warp scan of the lanes' counts.
+    // (one 16-byte load of their item ranks), gathers their class bytes into
+    // two words and turns them into 8-bit masks of keys above and at the cut
+    // (one multiply packs four bytes' low bits), so counting is two popcounts.
+    // Pass 1 counts the chunk; after one barrier every warp knows its chunk's
+    // output base, and pass 2 walks the chunk again, placing each lane's
+    // selected keys (those above the cut, and those at it while fewer than
+    // `need` came before) after an exclusive warp scan of the lanes' counts.
     const uint16_t *ki = a.key_item + (int64_t)bh * a.N;
     const bool vec8 = (((int64_t)bh * a.N) & 7) == 0;  // 16-byte aligned runs of eight ranks
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int chunk = (((a.N + nwarps - 1) / nwarps) + 255) & ~255;
     const int j_begin = min(a.N, warp * chunk), j_end = min(a.N, j_begin + chunk);
     __shared__ int wgt[32], weq[32];
-    // classes of keys j .. j+7: 2 above the cut, 1 at it, 0 below (or past the chunk)
-    auto classes8 = [&](int j, uint8_t (&k)[8]) {
+    // bit b of the result = bit `sh` of byte b of x (b < 4)
+    auto pack4 = [](uint32_t x, int sh) { return (((x >> sh) & 0x01010101u) * 0x01020408u) >> 24 & 0xfu; };
+    // masks of keys j .. j+7 above (bits of *ab) and at (*at) the cut; keys past the chunk are below
+    auto masks8 = [&](int j, uint32_t &ab, uint32_t &at) {
+        uint32_t lo, hi;
         if (vec8 && j + 8 <= j_end) {
             const uint4 w = *reinterpret_cast<const uint4 *>(ki + j);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int t = 0; t < 8; ++t) k[t] = class_of((ws[t >> 1] >> (16 * (t & 1))) & 0xffffu);
+            lo = (uint32_t)cls[w.x & 0xffffu] | (uint32_t)cls[w.x >> 16] << 8 | (uint32_t)cls[w.y & 0xffffu] << 16 |
+                 (uint32_t)cls[w.y >> 16] << 24;
+            hi = (uint32_t)cls[w.z & 0xffffu] | (uint32_t)cls[w.z >> 16] << 8 | (uint32_t)cls[w.w & 0xffffu] << 16 |
+                 (uint32_t)cls[w.w >> 16] << 24;
         } else {
+            lo = hi = 0u;
 #pragma unroll
-            for (int t = 0; t < 8; ++t) k[t] = j + t < j_end ? class_of(ki[j + t]) : 0;
+            for (int t = 0; t < 4; ++t) {
+                if (j + t < j_end) lo |= (uint32_t)cls[ki[j + t]] << (8 * t);
+                if (j + 4 + t < j_end) hi |= (uint32_t)cls[ki[j + 4 + t]] << (8 * t);
+            }
         }
+        ab = pack4(lo, 1) | pack4(hi, 1) << 4;
+        at = pack4(lo, 0) | pack4(hi, 0) << 4;
     };
     int g_cnt = 0, e_cnt = 0;
     for (int j0 = j_begin; j0 < j_end; j0 += 256) {
-        uint8_t k[8];
-        classes8(j0 + 8 * lane, k);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            g_cnt += k[t] == 2;
-            e_cnt += k[t] == 1;
-        }
+        uint32_t ab, at;
+        masks8(j0 + 8 * lane, ab, at);
+        g_cnt += __popc(ab);
+        e_cnt += __popc(at);
     }
     for (int o = 16; o > 0; o >>= 1) {
         g_cnt += __shfl_xor_sync(0xffffffffu, g_cnt, o);
@@ -908,14 +910,9 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
     int *stage = reinterpret_cast<int *>(S.met) + warp * 256;
     for (int j0 = j_begin; j0 < j_end; j0 += 256) {
         const int j = j0 + 8 * lane;
-        uint8_t k[8];
-        classes8(j, k);
-        unsigned lg = 0, le = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            lg += k[t] == 2;
-            le += k[t] == 1;
-        }
+        uint32_t ab, at;
+        masks8(j, ab, at);
+        const unsigned lg = __popc(ab), le = __popc(at);
         // exclusive scan of the lanes' (above, at) counts, packed in one word
         const unsigned packed = lg | (le << 16);
         unsigned incl = packed;
@@ -926,18 +923,26 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
         }
         const unsigned tot = __shfl_sync(0xffffffffu, incl, 31);
         const unsigned ex = incl - packed;
-        // Output slot of a selected key = selected keys before it: keys above
-        // the cut, plus keys at it up to `need`.  The step's selected keys
-        // land in this warp's staging row in order, then go out as coalesced
-        // 128-byte stores.
+        // output slot of a selected key = selected keys before it
         const unsigned base = g + min(e, (unsigned)need);  // selected keys before this step
-        unsigned gl = g + (ex & 0xffffu), el = e + (ex >> 16);
+        const unsigned gl = g + (ex & 0xffffu), el = e + (ex >> 16);
+        uint32_t sel = ab;
+        if (el < (unsigned)need) {
+            if (el + le <= (unsigned)need) {
+                sel |= at;
+            } else {  // the lane where the keys at the cut run out
+                uint32_t m = at;
+                for (unsigned k = el; k < (unsigned)need; ++k) {
+                    sel |= m & (0u - m);
+                    m &= m - 1u;
+                }
+            }
+        }
         unsigned pos = gl + min(el, (unsigned)need) - base;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const bool sel = k[t] == 2 || (k[t] == 1 && el < (unsigned)need);
-            if (k[t] == 1) ++el;
-            if (sel) stage[pos++] = j + t;
+        while (sel) {
+            const int t = __ffs(sel) - 1;
+            sel &= sel - 1u;
+            stage[pos++] = j + t;
         }
         g += tot & 0xffffu;
         e += tot >> 16;
@@ -954,6 +959,8 @@ __global__ void __launch_bounds__(kSelThreads) emit_kernel(SelArgs a, const int3
 // dynamic shared memory of topp_kernel and emit_kernel: the table row and a
 // 64 KB region (cached order keys, or item class bytes)
 static size_t sel_smem(int Csum) { return (size_t)((Csum + 3) & ~3) * sizeof(float) + (size_t)kItemCache * 4; }
+// emit_kernel also keeps a class byte per item after the region
+static size_t emit_smem(int Csum) { return sel_smem(Csum) + (size_t)kItemCache; }
 
 cudaError_t select_configure()
 {
@@ -965,7 +972,7 @@ cudaError_t select_configure()
     if (el != cudaSuccess) return el;
     const int max_csum = kMaxBlocks + 2 > 3 * kMaxClusters ? kMaxBlocks + 2 : 3 * kMaxClusters;
     cudaError_t e = cudaFuncSetAttribute(emit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sel_smem(max_csum));
+                                         (int)emit_smem(max_csum));
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(eg_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(3 * kMaxClusters * sizeof(float)));
@@ -1015,7 +1022,7 @@ void launch_topk(const int32_t *sizes, const int32_t *r, int32_t *n_out, int32_t
 void launch_emit(const SelArgs &a, const int32_t *n_in, const long long *offsets, const ClusterCut *cuts,
                  const int32_t *coarse_hist, int32_t *indices, cudaStream_t st)
 {
-    emit_kernel<<<dim3(a.Cq, a.BH), kSelThreads, sel_smem(a.Ct + a.Ch + a.Cw), st>>>(a, n_in, offsets, cuts,
+    emit_kernel<<<dim3(a.Cq, a.BH), kSelThreads, emit_smem(a.Ct + a.Ch + a.Cw), st>>>(a, n_in, offsets, cuts,
                                                                                   coarse_hist, indices);
     count_launches(1);
 }
