@@ -34,6 +34,7 @@ struct SelArgs {
     float top_p, inv_sqrt_d;
     int k_min;
     int whole_items;          // block mode: the cut takes every key tied at the cut score
+    int entropy;              // EG-Sparse: topp_kernel also records each row's entropy and ln Z
     int32_t *err;             // device error word
 };
 
@@ -176,6 +177,7 @@ struct SelShared {
     int coarse;  // the coarse bucket being refined (-1: none)
     unsigned long long above_met, run_met, bucket_met, new_above_met;
     int above_cnt, run_cnt, bucket_cnt, new_above_cnt, bucket;
+    int nlist;  // refine: items gathered from the coarse bucket
 };
 
 __device__ __forceinline__ float item_score(const float *L, int id, int Ch, int Cw, int Ct)
@@ -313,16 +315,81 @@ __device__ bool refine_pass(SelShared &S, const ItemKeys &K, const int32_t *cnts
 
 // After the coarse bucket is chosen (S.coarse, S.above_*): the exact order
 // key of the cut and the number of keys taken (-1 if the invariant broke,
-// which exact integer metrics rule out).
+// which exact integer metrics rule out).  The coarse bucket's items are
+// gathered first (key, count, metric; at most kRefineList of them, in the
+// select's bucket arrays, free by then): each gathered item then sums the
+// metric and count of the gathered items with a larger key and with its own
+// key, and the key where the running metric reaches the target is the cut,
+// exactly as the radix passes would find it.  A fuller bucket takes three
+// radix passes (11/11/10 bits of the order key) over every item instead.
+constexpr int kRefineList = 1024;
+
 __device__ int refine(SelShared &S, const ItemKeys &K, const int32_t *cnts, int n_items, const CoarseMap &cm,
                       float smax, float inv_sqrt_d, bool by_mass, unsigned long long target, uint32_t *cut_key,
                       int *need_at_cut, bool whole = false)
 {
-    if (threadIdx.x == 0) S.prefix = 0u;
+    static_assert(kBuckets >= 2 * kRefineList, "the gathered items live in the bucket arrays");
+    unsigned long long *lw = S.met;                                         // metric
+    uint32_t *lk = reinterpret_cast<uint32_t *>(S.met + kRefineList);      // order key
+    int *lc = S.cnt;                                                        // key count
+    if (threadIdx.x == 0) {
+        S.nlist = 0;
+        S.bucket = -1;
+        S.prefix = 0u;
+    }
     __syncthreads();
-    if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 21, 11)) return -1;
-    if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 10, 11)) return -1;
-    if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 0, 10)) return -1;
+    const int cb = S.coarse;
+    for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+        const uint32_t u = K(i);
+        const float sc = key_score(u);
+        if (cm(sc) != cb) continue;
+        const int slot = atomicAdd(&S.nlist, 1);
+        if (slot < kRefineList) {
+            lk[slot] = u;
+            lc[slot] = cnts[i];
+            lw[slot] = by_mass ? (unsigned long long)cnts[i] * item_mass(sc, smax, inv_sqrt_d)
+                               : (unsigned long long)cnts[i];
+        }
+    }
+    __syncthreads();
+    const int m = S.nlist;
+    if (m <= kRefineList) {
+        for (int p = threadIdx.x; p < m; p += blockDim.x) {
+            const uint32_t u = lk[p];
+            unsigned long long wg = 0ull, we = 0ull;
+            int cg = 0, ce = 0;
+            for (int q = 0; q < m; ++q) {
+                const uint32_t v = lk[q];
+                if (v > u) {
+                    wg += lw[q];
+                    cg += lc[q];
+                } else if (v == u) {
+                    we += lw[q];
+                    ce += lc[q];
+                }
+            }
+            const unsigned long long before = S.above_met + wg;
+            if (before < target && target <= before + we) {  // every item of the cut key writes the same
+                S.bucket = 0;
+                S.prefix = u;
+                S.bucket_met = we;
+                S.bucket_cnt = ce;
+                S.new_above_met = before;
+                S.new_above_cnt = S.above_cnt + cg;
+            }
+        }
+        __syncthreads();
+        if (S.bucket < 0) return -1;
+        if (threadIdx.x == 0) {
+            S.above_met = S.new_above_met;
+            S.above_cnt = S.new_above_cnt;
+        }
+        __syncthreads();
+    } else {
+        if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 21, 11)) return -1;
+        if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 10, 11)) return -1;
+        if (!refine_pass(S, K, cnts, n_items, cm, smax, inv_sqrt_d, by_mass, target, 0, 10)) return -1;
+    }
     // every key in the final bucket has the same score, hence the same metric
     const unsigned long long per = S.bucket_met / (unsigned long long)S.bucket_cnt;
     const unsigned long long rest = target - S.above_met;
@@ -405,10 +472,12 @@ __global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r
             const unsigned long long w = (unsigned long long)cnts[i] * item_mass(sc, smax, a.inv_sqrt_d);
             atomicAdd(&S.met[b], w);
             wsum += w;
-            const float x = (sc - smax) * a.inv_sqrt_d;
-            const double e = (double)cnts[i] * (double)expf(x);
-            zs += e;
-            as += e * (double)x;
+            if (a.entropy) {
+                const float x = (sc - smax) * a.inv_sqrt_d;
+                const double e = (double)cnts[i] * (double)expf(x);
+                zs += e;
+                as += e * (double)x;
+            }
         }
     }
     for (int o = 16; o > 0; o >>= 1) {
@@ -459,8 +528,8 @@ __global__ void __launch_bounds__(kSelThreads) topp_kernel(SelArgs a, int32_t *r
             Z += S.dz[w];
             A += S.da[w];
         }
-        cut.lnz = sel && Z > 0.0 ? (float)log(Z) : 0.f;
-        cut.ent = sel && Z > 0.0 ? (float)(log(Z) - A / Z) : 0.f;
+        cut.lnz = a.entropy && sel && Z > 0.0 ? (float)log(Z) : 0.f;
+        cut.ent = a.entropy && sel && Z > 0.0 ? (float)(log(Z) - A / Z) : 0.f;
         cut.pad = 0;
         cuts[bhc] = cut;
     }
@@ -1061,6 +1130,7 @@ void run_selection(const float *lut, const int32_t *codes, const int32_t *item_i
     a.inv_sqrt_d = inv_sqrt_d;
     a.k_min = k_min;
     a.whole_items = whole_items;
+    a.entropy = (eg_tau > 0.f && top_p < 1.0f) ? 1 : 0;
     a.err = err;
     ClusterCut *cuts = reinterpret_cast<ClusterCut *>(state);
     int32_t *coarse_hist = reinterpret_cast<int32_t *>(cuts + (int64_t)BH * Cq);
