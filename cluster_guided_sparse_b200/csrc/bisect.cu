@@ -11,11 +11,21 @@
 // depth-first, child 0 first, which is the order of the member array after
 // the last level.
 //
-// One CTA per node per level.  delta is formed in fp64 and the member sums
-// are exact in fp64 (bf16 inputs), so the split agrees with an fp64
-// evaluation except at ties below 1e-15.  The median cut is a radix select on
-// the order-preserving 64-bit image of delta, and the children are written by
-// a stable partition (a packed block scan per 1024-member tile).
+// delta is formed in fp64 (dims in order) and the member sums are exact in
+// fp64 (bf16 inputs), so the split agrees with an fp64 evaluation except at
+// ties below 1e-15.  The median cut is an exact select on the order-preserving
+// 64-bit image of delta (equal keys taken in member order): min and max, a
+// histogram of equal-width value buckets (the bucket is a non-decreasing
+// function of delta), then the crossing bucket's keys alone, ranked by one
+// warp when there are at most 32 of them and by a radix select otherwise (a
+// radix select over all members when the bucket is too full).  Members go to
+// their side by a plain comparison unless some keys at the cut are left out;
+// the children are written by a stable partition (a block scan per tile).
+// Nodes of 2048 rows and more run each round as four kernels over all
+// members (delta, cut, side sums, means); smaller nodes as one CTA per node
+// with every round inside.  The queries' and the keys' row sets of a call are
+// bisected together (2*BH row sets), so the top levels' few nodes fill more
+// of the GPU.
 #include "common.cuh"
 
 namespace scope {
