@@ -13,9 +13,11 @@
 // A key's score depends only on its code triple (a_t, a_h, a_w), so the
 // selection runs over the distinct triples of a head, each weighted by how
 // many keys carry it (16 384 triples instead of 118 800 keys at 720p).  The
-// Top-p cut is a radix select over the order-preserving 32-bit image of the
-// score, carrying per-bucket key counts and softmax masses; masses are 64-bit
-// fixed point (2^40 units) so their sums are exact and order-free.
+// Top-p cut is an exact select over the order-preserving 32-bit image of the
+// score: a coarse histogram over the row's score range, then the crossing
+// bucket's triples gathered and ranked (radix passes when the bucket is
+// full), carrying key counts and softmax masses; masses are 64-bit fixed
+// point (2^40 units) so their sums are exact and order-free.
 #include "common.cuh"
 
 namespace scope {
