@@ -148,7 +148,7 @@ struct CoarseT {
     int nlist, bucket, below;
 };
 using CoarseShared = CoarseT<kCoarse, kCoarseCap>;  // top-level nodes (one CTA per node)
-using CoarseSmall = CoarseT<2048, 32>;             // nodes of up to 1024 rows
+using CoarseSmall = CoarseT<2048, 256>;            // nodes of up to 2048 rows
 
 // The exact cut among m <= 32 keys, by one warp: a lane's key is the cut when
 // fewer than k keys are below it and at least k are at or below it.
@@ -165,6 +165,30 @@ __device__ void small_select(BisectShared &S, const unsigned long long *list, in
         }
         const unsigned hit = __ballot_sync(0xffffffffu, lane < m && lt < k && k <= le);
         if (lane == __ffs(hit) - 1) {
+            S.prefix = u;
+            S.need = k - lt;
+            S.eq = le - lt;
+        }
+    }
+    __syncthreads();
+    c.key = S.prefix;
+    c.need = S.need;
+    c.eq = S.eq;
+}
+
+// The same for m <= a few hundred keys, block-wide: every key counts the keys
+// below it and at or below it.
+__device__ void block_rank_select(BisectShared &S, const unsigned long long *list, int m, int k, Cut &c)
+{
+    for (int p = threadIdx.x; p < m; p += blockDim.x) {
+        const unsigned long long u = list[p];
+        int lt = 0, le = 0;
+        for (int q = 0; q < m; ++q) {
+            const unsigned long long v = list[q];
+            lt += v < u ? 1 : 0;
+            le += v <= u ? 1 : 0;
+        }
+        if (lt < k && k <= le) {  // every key equal to the cut writes the same values
             S.prefix = u;
             S.need = k - lt;
             S.eq = le - lt;
@@ -242,6 +266,7 @@ __device__ void select_k_coarse(BisectShared &S, CoarseT<NB, CAP> &C, const doub
     }
     __syncthreads();
     if (m <= 32) small_select(S, C.list, m, k - below, c);
+    else if (m <= 512) block_rank_select(S, C.list, m, k - below, c);
     else radix_select(S, [&](int i) { return C.list[i]; }, m, k - below, c);
 }
 
