@@ -410,3 +410,43 @@ def test_second_batch_entry_stage_fed():
                           np.arange(w.c_q), tc)
         P.check_attention(qr, kr, v[b, h].double().numpy(), qlab, get, P.np64(o[b, h]), np.arange(0, N, 7))
     tc.assert_ok("batch 1 Top-p counts")
+
+
+# B > 1 through the ClusterAttention path: the bisection's 2*B*H row sets,
+# the grouped work items (unions and masks per (batch, head)) and the
+# compensation's virtual lists, checked on batch entry 1 against the oracle.
+def test_second_batch_entry_cluster_attention_compensated():
+    N, D, H, leaf = 4096, 64, 2, 64
+    w = synth.WORKLOADS["unstructured"].with_(B=2, N=N, D=D, H=H, d_split=(D, 0, 0), components=16, k_min=32,
+                                               config_id=195, c_q=N // leaf, c_sub=(N // leaf, 1, 1), top_p=0.8,
+                                               compensate=1, fixed_cluster_size=leaf)
+    q, k, v = synth.make_inputs(w)
+    qd, kd, vd = to_dev(q, k, v)
+    pl = plan_of(w, qd, kd)
+    o = scope.attn(qd, kd, vd, pl)
+    torch.cuda.synchronize()
+    pl.sync_status()
+    b, C = 1, N // leaf
+    rng = np.random.default_rng(11)
+    for h in range(H):
+        qr, kr = P.np64(pl.view("qr")[b, h]), P.np64(pl.view("kr")[b, h])
+        qlab = pl.view("q_labels")[b, h].cpu().numpy()
+        klab = pl.view("k_codes")[0, b, h].cpu().numpy()
+        for X, lab_gpu in ((qr, qlab), (kr, klab)):
+            lab, _, _ = oracle.bisect(X, leaf, w.iters)
+            assert (lab == lab_gpu).all(), f"bisection labels differ on {(lab != lab_gpu).sum()} rows"
+        get = lists_fn(pl, w, h, B=b)
+        # the grouped lists of flat head (b, h)
+        off = pl.view("offsets").cpu().numpy()
+        gn = pl.view("group_n")[b, h].cpu().numpy()
+        gidx = pl.view("group_indices")
+        bh, Lg = b * H + h, 256 // leaf
+        for g in range(C // Lg):
+            u = np.unique(np.concatenate([get(c) for c in range(g * Lg, (g + 1) * Lg)]))
+            start = int(off[bh * C + g * Lg])
+            assert int(gn[g]) == len(u) and (gidx[start:start + len(u)].cpu().numpy() == u).all(), (h, g)
+        rows = np.sort(rng.choice(N, 64, replace=False))
+        ref = np.stack([oracle.attention_rows_comp(qr[n:n + 1], kr, v[b, h].double().numpy(), get(qlab[n]), klab,
+                                                   1.0 / np.sqrt(D))[0] for n in rows])
+        max_abs, rel = P.attn_error(P.np64(o[b, h])[rows], ref)
+        assert max_abs <= P.ATTN_MAX_ABS and rel <= P.ATTN_REL_L2, f"compensated: max-abs {max_abs:.3g}, rel {rel:.3g}"
