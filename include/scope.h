@@ -226,7 +226,7 @@ typedef enum {
     SCOPE_VIEW_INDICES = 16,    /* i32  [capacity] selected keys, ascending per cluster */
     SCOPE_VIEW_ERROR = 17,      /* i32  [4] device error word              */
     SCOPE_VIEW_EG_ENTROPY = 18, /* f32  [B,H] EG-Sparse head entropy (eg_tau > 0) */
-    SCOPE_VIEW_EG_POOL = 19,    /* i32  [B,H] pool (group) of a routed head, -1 if not routed */
+    SCOPE_VIEW_EG_POOL = 19,    /* i32  [B,H] pool of a routed head (b * ceil(H/eg_group) + h/eg_group), -1 if not routed */
     SCOPE_VIEW_FIXUP = 20,      /* i32  [1] rows the last tensor-core query assignment sent to the fp64 re-check */
     /* ClusterAttention leaves of 32 or 64 queries: L = 256 / leaf consecutive
      * leaves form a group that the attention serves as one work item. */

@@ -85,3 +85,41 @@ def test_block_mode_argument_rules():
             scope.plan(qd, kd, *scope.make_params(w.with_(H=1), **bad))
     with pytest.raises(scope.ScopeError):
         scope.plan(qd, kd, *scope.make_params(w.with_(H=1), grid=(0, 0, 0)))
+
+
+def test_block_selection_second_batch_entry():
+    """B = 2: batch entry 1's block means, kept blocks and lists against the oracle."""
+    kind, dims = 3, (2, 4, 8)
+    w = synth.WORKLOADS["small"].with_(B=2, block_kind=kind, block_dims=dims, k_min=0, online_topk=0,
+                                       config_id=239)
+    q, k, v = synth.make_inputs(w)
+    qd, kd = q.to(DEV), k.to(DEV)
+    pl = scope.plan(qd, kd, *scope.make_params(w))
+    torch.cuda.synchronize()
+    pl.sync_status()
+    b, D = 1, w.D
+    scale = 1.0 / np.sqrt(D)
+    p32 = float(np.float32(w.top_p))
+    ids, nb = oracle.block_ids(w.grid, kind, dims)
+    bsizes = np.bincount(ids, minlength=nb).astype(np.int64)
+    off = pl.view("offsets").cpu().numpy()
+    idx = pl.view("indices")
+    ties = 0
+    for h in range(w.H):
+        assert (pl.view("k_codes")[0, b, h].cpu().numpy() == ids).all()
+        kbar = P.np64(pl.view("k_cent_t")[b, h])
+        ref = oracle.block_means(P.np64(pl.view("kr")[b, h]), ids, nb)
+        assert np.abs(kbar - ref).max() <= 1e-6 * max(1.0, np.abs(ref).max())
+        lut = pl.view("lut")[b, h].cpu().numpy()
+        n = pl.view("n")[b, h].cpu().numpy()
+        sizes = pl.view("q_sizes")[b, h].cpu().numpy()
+        for c in range(w.c_q):
+            if sizes[c] == 0:
+                continue
+            keep, m = oracle.block_select(lut[c, :nb].astype(np.float64), bsizes, p32, scale)
+            if m != int(n[c]):
+                ties += 1
+                continue
+            i0 = int(off[(b * w.H + h) * w.c_q + c])
+            assert (idx[i0:i0 + int(n[c])].cpu().numpy() == np.nonzero(keep[ids])[0]).all(), (h, c)
+    assert ties <= 2

@@ -122,3 +122,46 @@ def test_eg_off_and_all_routed():
     assert (allr.view("eg_pool") == 0).all()
     with pytest.raises(scope.ScopeError):
         base.view("eg_entropy")  # no routing in a plain plan
+
+
+def test_eg_pools_are_per_batch_entry():
+    """B = 2: each batch entry routes and pools its own heads; batch entry 1's
+    entropies, pools and pooled counts against the oracle."""
+    group = 4
+    w = synth.WORKLOADS["small"].with_(B=2, k_min=0, sigma=(0.1, 1.0), config_id=219)
+    q, k, v = synth.make_inputs(w)
+    qd, kd = q.to(DEV), k.to(DEV)
+    scale = 1.0 / np.sqrt(w.D)
+    p32 = float(np.float32(w.top_p))
+    probe = scope.plan(qd, kd, *scope.make_params(w.with_(eg_tau=1e-9, eg_group=group)))
+    srt = np.sort(probe.view("eg_entropy")[1].cpu().numpy())
+    i = int(np.argmax(np.diff(srt[1:-1]))) + 1
+    tau = float((srt[i] + srt[i + 1]) / 2)
+    wq = w.with_(eg_tau=tau, eg_group=group)
+    pl = scope.plan(qd, kd, *scope.make_params(wq))
+    torch.cuda.synchronize()
+    pl.sync_status()
+    b = 1
+    ent = pl.view("eg_entropy")[b].cpu().numpy()
+    pool = pl.view("eg_pool")[b].cpu().numpy()
+    sizes = pl.view("q_sizes")[b].cpu().numpy().astype(np.int64)
+    r = pl.view("r")[b].cpu().numpy()
+    scores = {}
+    for h in range(w.H):
+        lut = pl.view("lut")[b, h].cpu().numpy()
+        codes = [pl.view("k_codes")[s, b, h].cpu().numpy() for s in range(3)]
+        scores[h] = np.stack([P.scores_f32(lut[c], codes, w.c_sub) for c in range(w.c_q)])
+        assert abs(ent[h] - oracle.head_entropy(scores[h], sizes[h], scale)) <= 1e-5, h
+    routed = [h for h in range(w.H) if ent[h] < tau]
+    ngroups = (w.H + group - 1) // group  # pool ids are global: batch entry b owns b*ngroups ..
+    assert (pool == np.array([b * ngroups + h // group if h in routed else -1 for h in range(w.H)])).all()
+    for members in oracle.eg_route(list(ent), tau, group):
+        if not members:
+            continue
+        counts = oracle.pooled_topp(np.stack([scores[h] for h in members]), np.stack([sizes[h] for h in members]),
+                                    p32, scale)
+        dev = np.stack([r[h] for h in members]).astype(np.int64)
+        if not (dev == counts).all():
+            f = [_pool_mass([scores[h] for h in members], np.stack([sizes[h] for h in members]), x, scale)
+                 for x in (dev, counts)]
+            assert all(abs(x - p32) <= P.TIE_REL * p32 for x in f), f"pool {members}: beyond a near-tie"
